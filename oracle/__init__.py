@@ -1,0 +1,102 @@
+"""TEST INFRASTRUCTURE ONLY: the CPU oracle of the RWKV-4 WKV recurrence.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA path
+and imports nothing from it.
+
+* ``forward``       -- fp64 max-trick recurrence in plain C (``wkv4_oracle.c``).
+* ``decode``        -- repeated T=1 forward calls with the state carried in place.
+* ``brute``         -- the closed-form sums evaluated literally in 50-digit
+                       arithmetic (``oracle/brute.py``), for tiny inputs.
+
+The recurrence is the RWKV-4 WKV time mix whose fp32 per-channel numerator /
+denominator / max state with the max-trick is described in "RWKV in a
+self-built engine: a second non-attention paradigm (WKV/RNN)" (Methods table,
+"Precision"; Reproducibility / Provenance, "Implementation").
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wkv4_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "libwkv4_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (-O2, no fast-math) into oracle/_build."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                               "-pthread", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            d = ctypes.POINTER(ctypes.c_double)
+            lib.wkv4_oracle_forward.argtypes = [ctypes.c_int64] * 3 + [d] * 6 + [d, ctypes.c_int]
+            lib.wkv4_oracle_forward.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor of any float dtype -> exact fp64 widening
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def forward(k, v, w, u, state_in=None, *, want_y: bool = True, nthreads: int = 1):
+    """fp64 forward over k, v [B, T, C]; w, u [C]; state_in [3, B, C] or None.
+
+    Inputs are widened exactly to fp64 from whatever dtype they arrive in.
+    Returns (y [B,T,C] or None, state_out [3,B,C]) as fp64 numpy arrays.
+    """
+    k, v, w, u, s_in = _f64(k), _f64(v), _f64(w), _f64(u), _f64(state_in)
+    B, T, C = k.shape
+    assert v.shape == (B, T, C) and w.shape == (C,) and u.shape == (C,)
+    if s_in is not None:
+        assert s_in.shape == (3, B, C)
+    y = np.empty((B, T, C), dtype=np.float64) if want_y else None
+    s_out = np.empty((3, B, C), dtype=np.float64)
+    rc = _load().wkv4_oracle_forward(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(s_in),
+                                     _ptr(y), _ptr(s_out), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"wkv4_oracle_forward failed ({rc})")
+    return y, s_out
+
+
+def decode(k, v, w, u, state):
+    """One T=1 step over k, v [B, C]: returns (y [B,C], new state [3,B,C])."""
+    k, v = _f64(k), _f64(v)
+    y, s = forward(k[:, None, :], v[:, None, :], w, u, state)
+    return y[:, 0, :], s
+
+
+def empty_state(B: int, C: int) -> np.ndarray:
+    s = np.zeros((3, B, C), dtype=np.float64)
+    s[2] = -1e38
+    return s

@@ -1,0 +1,153 @@
+"""Seeded synthetic inputs for the RWKV-4 WKV forward and decode workloads.
+
+This module draws numbers and nothing else: it holds none of the WKV arithmetic,
+so both the CUDA path and the CPU oracle can take their inputs from it without
+sharing any of the method's code.
+
+Workloads (sizes of the RWKV-4 models the pages discuss):
+
+* ``tiny``                 B=1,  T=16,    C=768,  fp32 I/O, zero state.
+* ``rwkv4_169m_prefill``   B=8,  T=1024,  C=768,  fp16 I/O, random state
+  (RWKV-4-169m width; "RWKV in a self-built engine: a second non-attention
+  paradigm (WKV/RNN)", Methods table, "Model" and "Precision" rows).
+* ``rwkv4_14b_prefill``    B=4,  T=1024,  C=5120, bf16 I/O, zero state
+  (d_model 5120 and 1K context of "RWKV-4 14B", "Every architecture field").
+* ``decode_b256``          B=256, C=5120, T=1 per call for 1024 calls, bf16.
+* ``long_t65536``          B=1,  T=65536, C=2048, fp32 I/O, 0.1% of k set to +30.
+
+Recipe (the same for every workload; knobs per workload below):
+
+* ``rng = numpy.random.default_rng(seed)``; draw order: time_decay[C], u[C],
+  initial state (num[B,C], den[B,C], max[B,C]) when it is random, k[B,T,C],
+  v[B,T,C], then the spike positions.
+* ``N(0, s)`` names a normal of *variance* s (standard deviation sqrt(s)).
+* ``w = -exp(time_decay)`` is evaluated in fp64 and rounded to fp32; u is fp32.
+* k and v are drawn in fp64 and rounded to nearest-even into the I/O dtype
+  (bf16 through torch's CPU cast).
+* Spikes: exactly ``round(frac * B*T*C)`` distinct flat positions of k, drawn
+  without replacement, are *set* to the spike value.
+* Decode draws w, u from ``default_rng(seed)`` and each call's k, v from
+  ``default_rng([seed, step])``.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+import torch
+
+_TORCH_DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    T: int
+    C: int
+    dtype: str                     # "f32" | "f16" | "bf16": dtype of k, v and y
+    seed: int
+    k_var: float = 1.0
+    v_var: float = 1.0
+    td_range: tuple = (-6.0, 1.0)  # time_decay ~ U(lo, hi)
+    u_range: tuple = (-1.0, 1.0)   # u ~ U(lo, hi)
+    random_state: bool = False     # num ~ N(0,1), den ~ U(0.5,2), max ~ U(-2,2)
+    spike_frac: float = 0.0
+    spike_value: float = 30.0
+    steps: int = 1                 # decode workloads: number of T=1 calls
+
+    @property
+    def channel_steps(self) -> int:
+        return self.B * self.T * self.C * self.steps
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return _TORCH_DTYPES[self.dtype]
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", B=1, T=16, C=768, dtype="f32", seed=0),
+    "rwkv4_169m_prefill": Workload("rwkv4_169m_prefill", B=8, T=1024, C=768, dtype="f16",
+                                   seed=1, random_state=True),
+    "rwkv4_14b_prefill": Workload("rwkv4_14b_prefill", B=4, T=1024, C=5120, dtype="bf16",
+                                  seed=2, k_var=2.0),
+    "decode_b256": Workload("decode_b256", B=256, T=1, C=5120, dtype="bf16", seed=3,
+                            steps=1024),
+    "long_t65536": Workload("long_t65536", B=1, T=65536, C=2048, dtype="f32", seed=4,
+                            k_var=4.0, td_range=(-8.0, 2.0), u_range=(-3.0, 3.0),
+                            spike_frac=0.001, spike_value=30.0),
+}
+
+
+def workload(name: str, **overrides) -> Workload:
+    w = WORKLOADS[name]
+    return w.replace(**overrides) if overrides else w
+
+
+def _to_io(x: np.ndarray, dtype: str) -> torch.Tensor:
+    """Round fp64 samples to nearest-even in the I/O dtype."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64))
+    return t.to(_TORCH_DTYPES[dtype]).contiguous()
+
+
+def _draw_params(rng: np.random.Generator, wl: Workload):
+    td = rng.uniform(wl.td_range[0], wl.td_range[1], size=wl.C)
+    u = rng.uniform(wl.u_range[0], wl.u_range[1], size=wl.C)
+    w = torch.from_numpy((-np.exp(td)).astype(np.float32))
+    return w, torch.from_numpy(u.astype(np.float32))
+
+
+def forward_inputs(wl: Workload) -> dict:
+    """Inputs of one forward call: w[C], u[C] fp32; k, v [B,T,C] in the I/O
+    dtype; state_in [3,B,C] fp32 (planes num, den, max) or None for the zero
+    state."""
+    rng = np.random.default_rng(wl.seed)
+    w, u = _draw_params(rng, wl)
+    state = None
+    if wl.random_state:
+        num = rng.standard_normal((wl.B, wl.C))
+        den = rng.uniform(0.5, 2.0, size=(wl.B, wl.C))
+        mx = rng.uniform(-2.0, 2.0, size=(wl.B, wl.C))
+        state = torch.from_numpy(np.stack([num, den, mx]).astype(np.float32)).contiguous()
+    shape = (wl.B, wl.T, wl.C)
+    k = rng.standard_normal(shape) * math.sqrt(wl.k_var)
+    v = rng.standard_normal(shape) * math.sqrt(wl.v_var)
+    if wl.spike_frac > 0.0:
+        n = int(round(wl.spike_frac * k.size))
+        idx = rng.choice(k.size, size=n, replace=False)
+        k.reshape(-1)[idx] = wl.spike_value
+    return {"w": w, "u": u, "k": _to_io(k, wl.dtype), "v": _to_io(v, wl.dtype),
+            "state_in": state}
+
+
+def decode_params(wl: Workload):
+    """w[C], u[C] of a decode workload."""
+    rng = np.random.default_rng(wl.seed)
+    return _draw_params(rng, wl)
+
+
+def decode_step_inputs(wl: Workload, step: int):
+    """k, v [B,C] of decode call number ``step`` (freshly seeded per call)."""
+    rng = np.random.default_rng([wl.seed, step])
+    shape = (wl.B, wl.C)
+    k = rng.standard_normal(shape) * math.sqrt(wl.k_var)
+    v = rng.standard_normal(shape) * math.sqrt(wl.v_var)
+    return _to_io(k, wl.dtype), _to_io(v, wl.dtype)
+
+
+def custom(B: int, T: int, C: int, dtype: str = "f32", seed: int = 0, **kw) -> dict:
+    """Inputs of an arbitrary shape drawn with the same recipe."""
+    return forward_inputs(Workload("custom", B=B, T=T, C=C, dtype=dtype, seed=seed, **kw))
+
+
+def zero_state(B: int, C: int) -> torch.Tensor:
+    """The empty state: num = den = 0 and max = -1e38 (fp32)."""
+    s = torch.zeros((3, B, C), dtype=torch.float32)
+    s[2].fill_(-1e38)
+    return s
