@@ -1,0 +1,431 @@
+"""Throughput of the RWKV-4 WKV forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--variant auto|seq|scan|scan_ldg|step]
+
+A step is one wkv4_forward call (the whole hot path: load, chunk summaries,
+segment chaining, outputs, final state) over one batch of the workload,
+default ``rwkv4_169m_prefill`` (B=8, T=1024, C=768, fp16 k/v/y, random fp32
+state in and out).  Inputs are seeded synthetic data (rwkv_wkv_linear_b200.synth)
+resident in HBM; the timed steps rotate over enough input sets that their
+total exceeds 3x the L2 cache, so no step reads another step's data from L2.
+The K steps run as CUDA-graph replays of the public call; the device time of
+the region (CUDA events on the launching stream) is max-reduced over ranks.
+
+Under torchrun each rank processes its own batch (independent sequences, no
+collective on the data path): weak scaling.
+
+``--impl reference`` times the fp64 CPU oracle on the same workload instead
+(rank 0 only; other ranks exit).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "WKV-4 forward G channel-steps/s (B·T·C/s) and achieved HBM GB/s vs peak"
+UNIT = "G channel-steps/s"
+L2_BYTES = 126 * 1024 * 1024
+VARIANTS = {"auto": 0, "seq": 1, "scan": 2, "scan_ldg": 3, "step": 4}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="rwkv4_169m_prefill")
+    ap.add_argument("--variant", default="auto", choices=sorted(VARIANTS))
+    ap.add_argument("--graph-steps", type=int, default=500,
+                    help="forward calls captured per CUDA graph")
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=5)
+
+    def summary(self):
+        sm = []
+        mx = None
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def io_bytes(wl):
+    es = {"f32": 4, "f16": 2, "bf16": 2}[wl.dtype]
+    return wl.B * wl.T * wl.C * es
+
+
+def algorithmic_bytes(wl):
+    """k, v read + y written (I/O dtype) + state in (when given) and out (fp32
+    triples) + w, u (fp32)."""
+    state = 12 * wl.B * wl.C
+    return 3 * io_bytes(wl) + (state if wl.random_state else 0) + state + 8 * wl.C
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rwkv_wkv_linear_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, variant):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[f"{workload}/{variant}"]
+        if e["kernel_source_hash"] == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def cpu_baseline(wl, x):
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    oracle.forward(x["k"][:1, :8], x["v"][:1, :8], x["w"], x["u"], None, nthreads=cores)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward(x["k"], x["v"], x["w"], x["u"], x["state_in"], nthreads=cores)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if reps >= 3 and dt > 1.0 or dt > 20.0:
+            break
+    return {"value": wl.channel_steps * reps / dt / 1e9, "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"the whole workload ({wl.B}x{wl.T}x{wl.C}) x {reps} passes, fp64 C "
+                      f"recurrence, {cores} threads over channels"}
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from rwkv_wkv_linear_b200 import synth, wkv4
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wkv4.load()
+    variant = VARIANTS[args.variant]
+    wl = synth.workload(args.workload)
+    x = synth.forward_inputs(wl.replace(seed=wl.seed + 1000 * rank) if rank else wl)
+
+    per_set = 2 * io_bytes(wl) + io_bytes(wl) + 24 * wl.B * wl.C
+    nsets = max(2, -(-3 * L2_BYTES // per_set))
+    nsets = min(nsets, max(2, int(20e9 // per_set)))
+    w, u = x["w"].to(dev), x["u"].to(dev)
+    ks = [x["k"].to(dev) for _ in range(nsets)]
+    vs = [x["v"].to(dev) for _ in range(nsets)]
+    sis = [x["state_in"].to(dev) if x["state_in"] is not None else None for _ in range(nsets)]
+    ys = [torch.empty_like(ks[0]) for _ in range(nsets)]
+    sos = [torch.empty((3, wl.B, wl.C), dtype=torch.float32, device=dev) for _ in range(nsets)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        j = i % nsets
+        wkv4.forward(ks[j], vs[j], w, u, sis[j], y=ys[j], state_out=sos[j], variant=variant,
+                     stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+
+    K = args.steps
+    gsteps = max(1, min(args.graph_steps, K))
+    graphs = []
+
+    def capture(n, offset):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                step(offset + i)
+        return g
+
+    main_graph = capture(gsteps, 0)
+    nrep, rem = divmod(K, gsteps)
+    rem_graph = capture(rem, 0) if rem else None
+    with torch.cuda.stream(stream):  # upload the graphs (untimed)
+        main_graph.replay()
+        if rem_graph is not None:
+            rem_graph.replay()
+    stream.synchronize()
+
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
+    clocks.start()
+    time.sleep(0.2)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(nrep):
+            main_graph.replay()
+        if rem_graph is not None:
+            rem_graph.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    ms = start.elapsed_time(end)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    if wkv4.device_error() != 0:
+        raise RuntimeError("device-side wait ran out during the timed region")
+
+    # end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        kh, vh = x["k"].pin_memory(), x["v"].pin_memory()
+        sih = x["state_in"].pin_memory() if x["state_in"] is not None else None
+        yh = torch.empty_like(kh).pin_memory()
+        soh = torch.empty((3, wl.B, wl.C), dtype=torch.float32).pin_memory()
+        kd, vd, yd, sod = ks[0], vs[0], ys[0], sos[0]
+        sid = sis[0]
+
+        def e2e_step():
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            if sih is not None:
+                sid.copy_(sih, non_blocking=True)
+            wkv4.forward(kd, vd, w, u, sid, y=yd, state_out=sod, variant=variant, stream=stream)
+            yh.copy_(yd, non_blocking=True)
+            soh.copy_(sod, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, args.e2e_steps)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(n_e2e):
+                e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize()
+        t2 = torch.tensor([s2.elapsed_time(e2)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        h2d = 2 * io_bytes(wl) + (12 * wl.B * wl.C if sih is not None else 0)
+        d2h = io_bytes(wl) + 12 * wl.B * wl.C
+        e2e = {"value": world * wl.channel_steps * n_e2e / (float(t2.item()) / 1e3) / 1e9,
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": n_e2e}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        per_launch_s = ms / 1e3 / K
+        achieved = algorithmic_bytes(wl) / per_launch_s / 1e9
+        line = {
+            "metric": METRIC,
+            "value": world * wl.channel_steps * K / (ms / 1e3) / 1e9,
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms / K,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
+                       "io_dtype": wl.dtype, "state_in": "random" if wl.random_state else "none",
+                       "global_batch": wl.B * world, "seq_len": wl.T,
+                       "parallelism": f"independent sequences per rank (x{world})",
+                       "kernel": args.variant,
+                       "l2": f"inputs rotate over {nsets} sets ({nsets * per_set / 1e6:.0f} MB "
+                             f"> 3x L2)",
+                       "launch": f"CUDA graphs of {gsteps} calls, {nrep}+{1 if rem else 0} "
+                                 "replays (one untimed upload replay each)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "bytes_per_launch": algorithmic_bytes(wl),
+                         "traffic": recorded_traffic(wl.name, args.variant)},
+            "gpu_launches": K,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, x)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The fp64 CPU oracle timed on this host's cores, on a bounded sample of
+    the workload per step (all T steps of the first channels of the batch), so
+    that --warmup W --steps K ends within a few minutes."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from rwkv_wkv_linear_b200 import synth
+
+    wl = synth.workload(args.workload)
+    x = synth.forward_inputs(wl)
+    cores = len(os.sched_getaffinity(0))
+    BC = wl.B * wl.C
+    # calibrate: channel-steps per second of the oracle on this host
+    n_cal = min(BC, max(1, 2_000_000 // wl.T))
+    cal = _ref_sample(x, wl, n_cal)
+    t0 = time.perf_counter()
+    oracle.forward(*cal, nthreads=cores)
+    rate = n_cal * wl.T / max(time.perf_counter() - t0, 1e-6)
+    budget_s = 150.0 / max(1, args.steps + args.warmup)
+    n_ch = int(min(BC, max(1, budget_s * rate / wl.T)))
+    smp = _ref_sample(x, wl, n_ch)
+    for _ in range(args.warmup):
+        oracle.forward(*smp, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(*smp, nthreads=cores)
+    dt = time.perf_counter() - t0
+    value = n_ch * wl.T * args.steps / dt / 1e9
+    sample = (f"{n_ch} of {BC} channels x all {wl.T} steps per step (fp64 C recurrence, "
+              f"{cores} threads)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C, "io_dtype": wl.dtype},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _ref_sample(x, wl, n_ch):
+    """The first n_ch flat channels (b*C + c) of the workload as one batch row:
+    (k, v, w, u, state_in) fp64 arrays for oracle.forward."""
+    import numpy as np
+    BC = wl.B * wl.C
+    ch = np.arange(n_ch)
+    c = ch % wl.C
+    k = x["k"].double().numpy().transpose(1, 0, 2).reshape(wl.T, BC)[:, :n_ch]
+    v = x["v"].double().numpy().transpose(1, 0, 2).reshape(wl.T, BC)[:, :n_ch]
+    w = x["w"].double().numpy()[c]
+    u = x["u"].double().numpy()[c]
+    s = None
+    if x["state_in"] is not None:
+        s = np.ascontiguousarray(x["state_in"].double().numpy().reshape(3, BC)[:, None, :n_ch])
+    return (np.ascontiguousarray(k[None]), np.ascontiguousarray(v[None]), w, u, s)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,151 @@
+/*
+ * wkv4.h -- C ABI of the RWKV-4 WKV forward and decode step on NVIDIA B200 (sm_100a).
+ *
+ * The operation (per batch row b and channel c, independently):
+ *   with decay w = w_c (normally -exp(time_decay_c)) and bonus u = u_c,
+ *   wkv_t = ( sum_{i<t} e^{(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *         / ( sum_{i<t} e^{(t-1-i) w + k_i}     + e^{u + k_t}     ),
+ * i.e. the RWKV-4 time-mix recurrence, carried as a per-channel fp32
+ * (numerator, denominator, max) state with the max-trick: "RWKV in a
+ * self-built engine: a second non-attention paradigm (WKV/RNN)", abstract,
+ * Methods table ("Precision": WKV numerator/denominator/max state carried in
+ * fp32) and Reproducibility / Provenance ("Implementation").  That the state
+ * is first-class -- produced by one call and consumed by the next, tracked by
+ * the caller -- follows "An RNN that claims to match transformers, now in
+ * chatbot form" ("The interesting bit"; "Caveats").
+ *
+ * State layout: one fp32 buffer [3][B][C], planes (num a, den b, max p), C
+ * fastest, with true numerator A = a e^p and denominator D = b e^p (natural
+ * units).  The empty state is (0, 0, -1e38).  A state given on entry is the
+ * state after the previous call's last token: it enters output t with weight
+ * e^{t w}, so splitting T over two calls with the state carried gives the
+ * result of one call (to fp32 rounding).
+ *
+ * Tensor layout: k, v, y are [B][T][C] row-major (C fastest) in the I/O dtype;
+ * w, u are fp32 [C].  All pointers are DEVICE pointers owned by the caller;
+ * the library keeps none of them after the call returns.
+ *
+ * Calls are asynchronous on `stream` (NULL = the legacy default stream) and
+ * return a status without synchronising.  Pointers need no particular
+ * alignment: misaligned or odd-C inputs take a slower element-wise path.
+ * NaN / Inf inputs propagate unchecked.  Distinct calls may run concurrently
+ * on different streams.
+ */
+#ifndef WKV4_H
+#define WKV4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define WKV4_API __attribute__((visibility("default")))
+#else
+#define WKV4_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* wkv4_stream_t; /* a cudaStream_t */
+
+/* I/O dtype of k, v and y.  w, u and the state are always fp32. */
+enum {
+    WKV4_F32 = 0,
+    WKV4_F16 = 1,
+    WKV4_BF16 = 2
+};
+
+/* status codes (0 = success, negative = error) */
+enum {
+    WKV4_OK = 0,
+    WKV4_ERR_ARG = -1,     /* a required pointer is NULL, or B/T/C < 0 */
+    WKV4_ERR_DTYPE = -2,   /* dtype is not one of WKV4_F32/F16/BF16 */
+    WKV4_ERR_ALIAS = -3,   /* y or the output state overlaps an input it must not */
+    WKV4_ERR_CUDA = -4,    /* a CUDA runtime call or kernel launch failed */
+    WKV4_ERR_TIMEOUT = -5, /* a bounded device-side wait ran out (see wkv4_device_error) */
+    WKV4_ERR_ALLOC = -6,   /* stream-ordered scratch allocation failed */
+    WKV4_ERR_VARIANT = -7  /* unknown kernel variant */
+};
+
+/*
+ * Forward over T time steps (prefill).
+ *   B, T, C     batch rows, time steps, channels.  B == 0 or C == 0: no-op.
+ *               T == 0: state_out <- state_in (or the empty state).
+ *   w, u        [C] fp32 decay (w = -exp(time_decay), supplied by the caller)
+ *               and bonus, both in natural-log units.
+ *   k, v        [B][T][C] in `dtype`.
+ *   state_in    [3][B][C] fp32, or NULL for the empty state.
+ *   y           [B][T][C] in `dtype`, written with round-to-nearest-even.
+ *               Must not overlap k, v, w, u, state_in or state_out.
+ *   state_out   [3][B][C] fp32 state after the last step, or NULL.  May equal
+ *               state_in exactly (in-place update); any other overlap with an
+ *               input is WKV4_ERR_ALIAS.
+ *   stream      CUDA stream of the call.
+ *   dtype       WKV4_F32, WKV4_F16 or WKV4_BF16.
+ * Scratch: for long T the forward needs a small stream-ordered scratch
+ * buffer (per-segment summaries), taken from a library-owned CUDA memory pool
+ * on `stream` and returned to it on `stream`; WKV4_ERR_ALLOC if that fails.
+ * Returns WKV4_OK or an error code; a device-side wait that ran out is
+ * reported by wkv4_device_error().
+ */
+WKV4_API int wkv4_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                 const void* k, const void* v, const float* state_in, void* y,
+                 float* state_out, wkv4_stream_t stream, int dtype);
+
+/* Kernel choices of wkv4_forward_variant (for tests and tuning). */
+enum {
+    WKV4_KERNEL_AUTO = 0,     /* what wkv4_forward picks */
+    WKV4_KERNEL_SEQ = 1,      /* channel-parallel, sequential over T, TMA-staged time tiles */
+    WKV4_KERNEL_SCAN = 2,     /* chunked scan over (channel tile x time segment), TMA loads */
+    WKV4_KERNEL_SCAN_LDG = 3, /* the chunked scan with element-wise loads (any alignment) */
+    WKV4_KERNEL_STEP = 4      /* exact per-step max-trick, one thread per channel (any T) */
+};
+
+/* wkv4_forward with an explicit kernel choice.  SEQ and SCAN need TMA
+ * alignment (16-byte aligned k, v and y, and C * sizeof(dtype) a multiple of
+ * 16); when it is not met both run as SCAN_LDG.  AUTO and T == 1 run the
+ * decode-step kernel; an explicit choice runs that kernel for any T >= 1.
+ * Unknown variant: WKV4_ERR_VARIANT. */
+WKV4_API int wkv4_forward_variant(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                         const void* k, const void* v, const float* state_in, void* y,
+                         float* state_out, wkv4_stream_t stream, int dtype, int variant);
+
+/*
+ * One decode step (T = 1) for B sequences, updating the state in place.
+ *   w, u     [C] fp32.
+ *   k, v     [B][C] in `dtype`.
+ *   state    [3][B][C] fp32, read and overwritten (RNN mode: "An RNN that
+ *            claims to match transformers, now in chatbot form").
+ *   y        [B][C] in `dtype`; must not overlap k, v, w, u or state.
+ * Equal, bit for bit, to wkv4_forward with T = 1 and state_in == state_out.
+ */
+WKV4_API int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float* u, const void* k,
+                     const void* v, float* state, void* y, wkv4_stream_t stream, int dtype);
+
+/* Bytes of stream-ordered scratch wkv4_forward_variant would take for this
+ * shape (0 when none), written to *bytes.  Host-only, no CUDA call. */
+WKV4_API int wkv4_forward_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype, int variant,
+                               size_t* bytes);
+
+/*
+ * Device-side error word of the current device (bit 0: a look-back wait ran
+ * out; bit 1: a TMA completion wait ran out).  Synchronises the device, reads
+ * the word, and clears it when `reset` is non-zero.  Returns WKV4_OK when the
+ * word is zero, WKV4_ERR_TIMEOUT when a wait ran out, WKV4_ERR_CUDA when the
+ * read itself failed.
+ */
+WKV4_API int wkv4_device_error(int reset);
+
+/* Static description of a status code. */
+WKV4_API const char* wkv4_status_string(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+WKV4_API int wkv4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV4_H */

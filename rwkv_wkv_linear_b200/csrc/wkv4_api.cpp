@@ -1,0 +1,308 @@
+// C ABI of the RWKV-4 WKV forward / decode step: argument checks, kernel
+// choice, TMA descriptors and stream-ordered scratch.  Every step of the
+// computation runs in the kernels of wkv4_kernels.cu; nothing here computes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <chrono>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <random>
+
+#include "../../include/wkv4.h"
+#include "wkv4_internal.h"
+
+namespace {
+
+using wkv4::FwdArgs;
+
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------------ helpers
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+
+Range range_of(const void* p, uint64_t bytes) {
+    const uintptr_t lo = (uintptr_t)p;
+    return {lo, lo + (uintptr_t)bytes};
+}
+
+bool overlap(Range a, Range b) {
+    if (a.lo == 0 || b.lo == 0 || a.lo == a.hi || b.lo == b.hi) return false;
+    return a.lo < b.hi && b.lo < a.hi;
+}
+
+bool is_aligned(const void* p, size_t n) { return p == nullptr || ((uintptr_t)p % n) == 0; }
+
+// Driver entry point of cuTensorMapEncodeTiled, fetched once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// 3-D map over a [B][T][C] tensor (dims innermost first: C, T, B) with a
+// box of box_c channels x box_t steps x 1 batch row; out-of-range elements
+// read as zero and are skipped on store.
+bool encode_btc(CUtensorMap* map, const void* ptr, int dtype, int64_t B, int64_t T, int64_t C,
+                int box_c, int box_t) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const size_t es = wkv4::dtype_size(dtype);
+    const CUtensorMapDataType dt = dtype == WKV4_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : dtype == WKV4_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)(C * es), (cuuint64_t)(T * C * es)};
+    const cuuint32_t box[3] = {(cuuint32_t)box_c, (cuuint32_t)box_t, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// TMA needs 16-byte aligned bases and row strides that are multiples of 16 bytes.
+bool tma_eligible(const FwdArgs& a) {
+    const size_t es = wkv4::dtype_size(a.dtype);
+    return (a.C * (int64_t)es) % 16 == 0 && is_aligned(a.k, 16) && is_aligned(a.v, 16) &&
+           is_aligned(a.y, 16) && a.T < (1ll << 31) && a.C < (1ll << 31) && a.B < (1ll << 31);
+}
+
+// Per-call epoch that tags the scan's cross-CTA flags, so stale flags left in
+// reused scratch memory never match.  Starts at a random point.
+std::atomic<unsigned long long>& epoch_counter() {
+    static std::atomic<unsigned long long> ctr{[] {
+        std::random_device rd;
+        unsigned long long x = ((unsigned long long)rd() << 32) ^ rd() ^
+                               (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+        return (x & ((1ull << 40) - 1)) + 1;
+    }()};
+    return ctr;
+}
+
+// Library-owned memory pool per device (release threshold: keep everything),
+// so stream-ordered scratch is recycled without returning to the driver.
+cudaMemPool_t device_pool(int dev) {
+    static cudaMemPool_t pools[kMaxDevices] = {};
+    static std::mutex mu;
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props;
+        std::memset(&props, 0, sizeof(props));
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+        unsigned long long keep = ~0ull;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        pools[dev] = pool;
+    }
+    return pools[dev];
+}
+
+int alloc_scratch(void** ptr, size_t bytes, cudaStream_t stream) {
+    *ptr = nullptr;
+    if (bytes == 0) return WKV4_OK;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return WKV4_ERR_CUDA;
+    cudaError_t e;
+    if (cap != cudaStreamCaptureStatusNone) {
+        e = cudaMallocAsync(ptr, bytes, stream);  // becomes a graph memory node
+    } else {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return WKV4_ERR_CUDA;
+        cudaMemPool_t pool = device_pool(dev);
+        if (!pool) return WKV4_ERR_ALLOC;
+        e = cudaMallocFromPoolAsync(ptr, bytes, pool, stream);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return WKV4_ERR_ALLOC;
+    }
+    return WKV4_OK;
+}
+
+int check_common(int64_t B, int64_t T, int64_t C, int dtype) {
+    if (B < 0 || T < 0 || C < 0) return WKV4_ERR_ARG;
+    if (dtype != WKV4_F32 && dtype != WKV4_F16 && dtype != WKV4_BF16) return WKV4_ERR_DTYPE;
+    return WKV4_OK;
+}
+
+int check_alias(const FwdArgs& a) {
+    const size_t es = wkv4::dtype_size(a.dtype);
+    const uint64_t io = (uint64_t)a.B * a.T * a.C * es;
+    const uint64_t st = (uint64_t)3 * a.B * a.C * 4;
+    const Range ry = range_of(a.y, io), rk = range_of(a.k, io), rv = range_of(a.v, io);
+    const Range rw = range_of(a.w, a.C * 4), ru = range_of(a.u, a.C * 4);
+    const Range rsi = range_of(a.state_in, st), rso = range_of(a.state_out, st);
+    if (overlap(ry, rk) || overlap(ry, rv) || overlap(ry, rw) || overlap(ry, ru) ||
+        overlap(ry, rsi) || overlap(ry, rso))
+        return WKV4_ERR_ALIAS;
+    if (overlap(rso, rk) || overlap(rso, rv) || overlap(rso, rw) || overlap(rso, ru))
+        return WKV4_ERR_ALIAS;
+    if (overlap(rso, rsi) && a.state_in != a.state_out) return WKV4_ERR_ALIAS;
+    return WKV4_OK;
+}
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return WKV4_OK;
+    cudaGetLastError();
+    return WKV4_ERR_CUDA;
+}
+
+int run_scan(const FwdArgs& a, bool want_tma) {
+    const bool tma = want_tma && tma_eligible(a);
+    CUtensorMap tk, tv, ty;
+    if (tma) {
+        const wkv4::Geom g = wkv4::scan_geom(a.dtype);
+        if (!encode_btc(&tk, a.k, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t) ||
+            !encode_btc(&tv, a.v, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t) ||
+            !encode_btc(&ty, a.y, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t))
+            return WKV4_ERR_CUDA;
+    }
+    void* scratch = nullptr;
+    const size_t bytes = wkv4::scan_scratch_bytes(a.B, a.T, a.C, a.dtype);
+    int rc = alloc_scratch(&scratch, bytes, a.stream);
+    if (rc != WKV4_OK) return rc;
+    const unsigned long long epoch = epoch_counter().fetch_add(1) & ((1ull << 62) - 1);
+    rc = cuda_status(wkv4::launch_scan(a, tma ? &tk : nullptr, tma ? &tv : nullptr,
+                                       tma ? &ty : nullptr, scratch, epoch));
+    if (scratch) {
+        const int rc2 = cuda_status(cudaFreeAsync(scratch, a.stream));
+        if (rc == WKV4_OK) rc = rc2;
+    }
+    return rc;
+}
+
+int run_seq(const FwdArgs& a) {
+    if (!tma_eligible(a) || !is_aligned(a.y, 16)) return run_scan(a, false);
+    const wkv4::Geom g = wkv4::seq_geom(a.dtype);
+    CUtensorMap tk, tv;
+    if (!encode_btc(&tk, a.k, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t) ||
+        !encode_btc(&tv, a.v, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t))
+        return WKV4_ERR_CUDA;
+    return cuda_status(wkv4::launch_seq(a, &tk, &tv));
+}
+
+// Kernel choice of wkv4_forward.  The sequential kernel needs enough channel
+// groups to fill the SMs on its own; otherwise the chunked scan splits T.
+int pick_variant(const FwdArgs& a) {
+    if (!tma_eligible(a)) return WKV4_KERNEL_SCAN_LDG;
+    if (a.B * a.C >= (1ll << 19) && a.T >= 64) return WKV4_KERNEL_SEQ;
+    return WKV4_KERNEL_SCAN;
+}
+
+int forward_impl(const FwdArgs& a, int variant) {
+    int rc = check_common(a.B, a.T, a.C, a.dtype);
+    if (rc != WKV4_OK) return rc;
+    if (variant < WKV4_KERNEL_AUTO || variant > WKV4_KERNEL_STEP) return WKV4_ERR_VARIANT;
+    if (a.B == 0 || a.C == 0) return WKV4_OK;
+    if (a.T == 0) {
+        rc = check_alias(a);
+        if (rc != WKV4_OK) return rc;
+        return cuda_status(wkv4::launch_copy_state(a));
+    }
+    if (!a.w || !a.u || !a.k || !a.v || !a.y) return WKV4_ERR_ARG;
+    rc = check_alias(a);
+    if (rc != WKV4_OK) return rc;
+    if (a.T == 1 && variant == WKV4_KERNEL_AUTO) return cuda_status(wkv4::launch_decode(a));
+    if (variant == WKV4_KERNEL_AUTO) variant = pick_variant(a);
+    switch (variant) {
+        case WKV4_KERNEL_SEQ: return run_seq(a);
+        case WKV4_KERNEL_SCAN: return run_scan(a, true);
+        case WKV4_KERNEL_SCAN_LDG: return run_scan(a, false);
+        default: return cuda_status(wkv4::launch_step(a));
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int wkv4_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const void* k,
+                 const void* v, const float* state_in, void* y, float* state_out,
+                 wkv4_stream_t stream, int dtype) {
+    return wkv4_forward_variant(B, T, C, w, u, k, v, state_in, y, state_out, stream, dtype,
+                                WKV4_KERNEL_AUTO);
+}
+
+int wkv4_forward_variant(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                         const void* k, const void* v, const float* state_in, void* y,
+                         float* state_out, wkv4_stream_t stream, int dtype, int variant) {
+    FwdArgs a{B, T, C, w, u, k, v, state_in, y, state_out, dtype, (cudaStream_t)stream};
+    return forward_impl(a, variant);
+}
+
+int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float* u, const void* k,
+                     const void* v, float* state, void* y, wkv4_stream_t stream, int dtype) {
+    int rc = check_common(B, 1, C, dtype);
+    if (rc != WKV4_OK) return rc;
+    if (B == 0 || C == 0) return WKV4_OK;
+    if (!w || !u || !k || !v || !y || !state) return WKV4_ERR_ARG;
+    FwdArgs a{B, 1, C, w, u, k, v, state, y, state, dtype, (cudaStream_t)stream};
+    rc = check_alias(a);
+    if (rc != WKV4_OK) return rc;
+    return cuda_status(wkv4::launch_decode(a));
+}
+
+int wkv4_forward_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype, int variant,
+                               size_t* bytes) {
+    if (!bytes) return WKV4_ERR_ARG;
+    *bytes = 0;
+    int rc = check_common(B, T, C, dtype);
+    if (rc != WKV4_OK) return rc;
+    if (variant < WKV4_KERNEL_AUTO || variant > WKV4_KERNEL_STEP) return WKV4_ERR_VARIANT;
+    if (B == 0 || C == 0 || T <= 1) return WKV4_OK;
+    if (variant == WKV4_KERNEL_STEP) return WKV4_OK;
+    if (variant == WKV4_KERNEL_AUTO || variant == WKV4_KERNEL_SEQ) {
+        // same decision as the call itself for aligned pointers
+        FwdArgs a{B, T, C, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dtype, nullptr};
+        const int pick = variant == WKV4_KERNEL_SEQ ? WKV4_KERNEL_SEQ : pick_variant(a);
+        if (pick == WKV4_KERNEL_SEQ && tma_eligible(a)) return WKV4_OK;
+    }
+    *bytes = wkv4::scan_scratch_bytes(B, T, C, dtype);
+    return WKV4_OK;
+}
+
+int wkv4_device_error(int reset) {
+    unsigned bits = 0;
+    if (wkv4::read_device_error(&bits, reset != 0) != cudaSuccess) {
+        cudaGetLastError();
+        return WKV4_ERR_CUDA;
+    }
+    return bits ? WKV4_ERR_TIMEOUT : WKV4_OK;
+}
+
+const char* wkv4_status_string(int status) {
+    switch (status) {
+        case WKV4_OK: return "ok";
+        case WKV4_ERR_ARG: return "invalid argument (NULL pointer or negative size)";
+        case WKV4_ERR_DTYPE: return "unknown dtype";
+        case WKV4_ERR_ALIAS: return "output overlaps an input";
+        case WKV4_ERR_CUDA: return "CUDA runtime error";
+        case WKV4_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+        case WKV4_ERR_ALLOC: return "scratch allocation failed";
+        case WKV4_ERR_VARIANT: return "unknown kernel variant";
+        default: return "unknown status";
+    }
+}
+
+int wkv4_version(void) { return 100; }
+
+}  // extern "C"

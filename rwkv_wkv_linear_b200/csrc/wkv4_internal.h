@@ -1,0 +1,52 @@
+// Host-side interface between the C ABI (wkv4_api.cpp) and the kernels
+// (wkv4_kernels.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace wkv4 {
+
+struct FwdArgs {
+    int64_t B, T, C;
+    const float* w;
+    const float* u;
+    const void* k;
+    const void* v;
+    const float* state_in;
+    void* y;
+    float* state_out;
+    int dtype;  // WKV4_F32 / WKV4_F16 / WKV4_BF16
+    cudaStream_t stream;
+};
+
+// Tile geometry of a kernel for one dtype: channels and steps per TMA box.
+struct Geom {
+    int box_c;      // channels per box (innermost TMA dimension)
+    int box_t;      // time steps per box
+    int threads;    // threads per CTA
+    size_t smem;    // dynamic shared memory per CTA (bytes)
+};
+
+Geom scan_geom(int dtype);
+Geom seq_geom(int dtype);
+size_t dtype_size(int dtype);
+
+// Scratch of the chunked scan: per (channel tile, time segment) a flag word
+// and two fp32 triples per channel (segment aggregate, inclusive prefix).
+size_t scan_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype);
+
+// Launchers.  Tensor maps are NULL for the element-wise (LDG) variants.
+cudaError_t launch_scan(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
+                        const CUtensorMap* ty, void* scratch, unsigned long long epoch);
+cudaError_t launch_seq(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv);
+cudaError_t launch_step(const FwdArgs& a);     // exact per-step kernel, any T >= 1
+cudaError_t launch_decode(const FwdArgs& a);   // T == 1, vectorised when aligned
+cudaError_t launch_copy_state(const FwdArgs& a);  // T == 0
+
+// Device error word of the current device (synchronous read; optional reset).
+cudaError_t read_device_error(unsigned* bits, bool reset);
+
+}  // namespace wkv4

@@ -1,0 +1,181 @@
+"""Python binding of the C ABI in include/wkv4.h (ctypes; argument marshalling only).
+
+Every step of the computation runs in the CUDA kernels of libwkv4.so; torch
+is used for device memory and streams.  There is no CPU fallback: when the
+library cannot be loaded every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwkv4.so")
+
+F32, F16, BF16 = 0, 1, 2
+KERNEL_AUTO, KERNEL_SEQ, KERNEL_SCAN, KERNEL_SCAN_LDG, KERNEL_STEP = 0, 1, 2, 3, 4
+
+STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_DTYPE", -3: "ERR_ALIAS", -4: "ERR_CUDA",
+          -5: "ERR_TIMEOUT", -6: "ERR_ALLOC", -7: "ERR_VARIANT"}
+
+_DTYPES = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+
+EXPORTS = ("wkv4_forward", "wkv4_forward_variant", "wkv4_decode_step",
+           "wkv4_forward_scratch_bytes", "wkv4_device_error", "wkv4_status_string",
+           "wkv4_version")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class Wkv4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what} failed: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libwkv4.so (raises OSError when it is missing: build it with
+    ``python -m rwkv_wkv_linear_b200._build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise OSError(f"{path} not found: build it with python -m rwkv_wkv_linear_b200._build")
+            lib = ctypes.CDLL(path)
+            i64, vp, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+            fwd = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32]
+            lib.wkv4_forward.argtypes = fwd
+            lib.wkv4_forward.restype = i32
+            lib.wkv4_forward_variant.argtypes = fwd + [i32]
+            lib.wkv4_forward_variant.restype = i32
+            lib.wkv4_decode_step.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp, vp, i32]
+            lib.wkv4_decode_step.restype = i32
+            lib.wkv4_forward_scratch_bytes.argtypes = [i64, i64, i64, i32, i32,
+                                                       ctypes.POINTER(ctypes.c_size_t)]
+            lib.wkv4_forward_scratch_bytes.restype = i32
+            lib.wkv4_device_error.argtypes = [i32]
+            lib.wkv4_device_error.restype = i32
+            lib.wkv4_status_string.argtypes = [i32]
+            lib.wkv4_status_string.restype = ctypes.c_char_p
+            lib.wkv4_version.argtypes = []
+            lib.wkv4_version.restype = i32
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().wkv4_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check_dev(name: str, t: Optional[torch.Tensor], dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def forward(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
+            state_in: Optional[torch.Tensor] = None, *, y: Optional[torch.Tensor] = None,
+            state_out: Optional[torch.Tensor] = None, want_state: bool = True,
+            variant: int = KERNEL_AUTO, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """wkv4_forward over k, v [B, T, C] (fp32/fp16/bf16); w, u [C] fp32;
+    state_in [3, B, C] fp32 or None.  Returns (y, state_out)."""
+    if k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("k and v must both be [B, T, C]")
+    B, T, C = k.shape
+    dt = _DTYPES.get(k.dtype)
+    if dt is None or v.dtype != k.dtype:
+        raise ValueError(f"unsupported dtype {k.dtype}/{v.dtype}")
+    for name, t in (("k", k), ("v", v)):
+        _check_dev(name, t)
+    _check_dev("w", w, torch.float32)
+    _check_dev("u", u, torch.float32)
+    _check_dev("state_in", state_in, torch.float32)
+    if w.shape != (C,) or u.shape != (C,):
+        raise ValueError("w and u must be [C]")
+    if state_in is not None and state_in.shape != (3, B, C):
+        raise ValueError("state_in must be [3, B, C]")
+    if y is None:
+        y = torch.empty_like(k)
+    _check_dev("y", y, k.dtype)
+    if state_out is None and want_state:
+        state_out = torch.empty((3, B, C), dtype=torch.float32, device=k.device)
+    _check_dev("state_out", state_out, torch.float32)
+    rc = load().wkv4_forward_variant(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(state_in),
+                                     _ptr(y), _ptr(state_out), _stream(stream), dt, int(variant))
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_forward")
+    return y, state_out
+
+
+def forward_raw(B: int, T: int, C: int, w, u, k, v, state_in, y, state_out, dtype: int,
+                variant: int = KERNEL_AUTO, stream=None) -> int:
+    """The C call with raw device addresses (ints or None); returns the status."""
+    return load().wkv4_forward_variant(B, T, C, w, u, k, v, state_in, y, state_out,
+                                       _stream(stream), dtype, int(variant))
+
+
+def decode_step(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
+                state: torch.Tensor, *, y: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """wkv4_decode_step: k, v [B, C]; state [3, B, C] fp32 updated in place.
+    Returns y [B, C]."""
+    if k.dim() != 2 or v.shape != k.shape:
+        raise ValueError("k and v must both be [B, C]")
+    B, C = k.shape
+    dt = _DTYPES.get(k.dtype)
+    if dt is None or v.dtype != k.dtype:
+        raise ValueError(f"unsupported dtype {k.dtype}/{v.dtype}")
+    for name, t in (("k", k), ("v", v)):
+        _check_dev(name, t)
+    _check_dev("w", w, torch.float32)
+    _check_dev("u", u, torch.float32)
+    _check_dev("state", state, torch.float32)
+    if state.shape != (3, B, C):
+        raise ValueError("state must be [3, B, C]")
+    if y is None:
+        y = torch.empty_like(k)
+    _check_dev("y", y, k.dtype)
+    rc = load().wkv4_decode_step(B, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(state), _ptr(y),
+                                 _stream(stream), dt)
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_decode_step")
+    return y
+
+
+def scratch_bytes(B: int, T: int, C: int, dtype: int, variant: int = KERNEL_AUTO) -> int:
+    n = ctypes.c_size_t(0)
+    rc = load().wkv4_forward_scratch_bytes(B, T, C, dtype, variant, ctypes.byref(n))
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_forward_scratch_bytes")
+    return int(n.value)
+
+
+def device_error(reset: bool = True) -> int:
+    """Status of the current device's error word (0, or -5 when a bounded
+    device-side wait ran out).  Synchronises the device."""
+    return int(load().wkv4_device_error(1 if reset else 0))
+
+
+def version() -> int:
+    return int(load().wkv4_version())

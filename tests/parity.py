@@ -1,7 +1,12 @@
 """Parity gates between the CUDA path and the fp64 oracle.
 
 y, fp32 I/O:       max |y - y_ref| <= 2e-5 * max|v|   (max over the call's v)
-y, fp16/bf16 I/O:  |y - y_ref| <= 2 ulp_dtype(|y_ref|) + 1e-3 |y_ref|, elementwise
+y, fp16/bf16 I/O:  |y - y_ref| <= 2 ulp_dtype(|y_ref|) + 1e-3 |y_ref| + 2e-5 * max|v|,
+                   elementwise: the outputs are computed in fp32 and then rounded, so
+                   the fp32 arithmetic's own allowance (the fp32 gate) is added to the
+                   rounding allowance; without it outputs near zero, where the fp32
+                   numerator cancels (|y| < 1e-4, in fp16's subnormal range), miss by
+                   an ulp or two of fp16
 state:             num and den are brought to a shared max m* = max(p, p_ref)
                    (x_hat = x * e^{p - m*}); den must agree to ``den_rtol``
                    relative and num/den (the running average) to
@@ -44,7 +49,8 @@ def y_violations(y, y_ref, v, dtype: str):
         bound = Y_ABS_F32 * float(np.max(np.abs(to_f64(v)))) if np.size(v) else 0.0
         bound = np.full_like(y_ref, bound)
     else:
-        bound = 2.0 * ulp(y_ref, dtype) + Y_REL_16 * np.abs(y_ref)
+        vmax = float(np.max(np.abs(to_f64(v)))) if np.size(v) else 0.0
+        bound = 2.0 * ulp(y_ref, dtype) + Y_REL_16 * np.abs(y_ref) + Y_ABS_F32 * vmax
     bad = ~(np.abs(y - y_ref) <= bound)  # NaN counts as a violation
     return bad, bound
 

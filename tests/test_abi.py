@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol that
+include/wkv4.h declares, and rejects bad arguments before touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from rwkv_wkv_linear_b200 import wkv4
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "wkv4.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"WKV4_API\s+[\w\s\*]*?\b(wkv4_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_symbols() == sorted(wkv4.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = wkv4.load()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings():
+    assert wkv4.version() == 100
+    for code in wkv4.STATUS:
+        assert wkv4.status_string(code)
+    assert wkv4.status_string(12345) == "unknown status"
+
+
+P = 0x7F0000000000  # fake device addresses: these calls must return before any CUDA call
+
+
+def _call(B=2, T=8, C=16, w=P, u=P + 0x1000, k=P + 0x10000, v=P + 0x20000, si=None,
+          y=P + 0x30000, so=None, dtype=wkv4.F32, variant=wkv4.KERNEL_AUTO):
+    return wkv4.load().wkv4_forward_variant(B, T, C, w, u, k, v, si, y, so, None, dtype, variant)
+
+
+def test_negative_sizes_are_rejected():
+    assert _call(B=-1) == -1
+    assert _call(T=-1) == -1
+    assert _call(C=-5) == -1
+
+
+def test_bad_dtype_and_variant():
+    assert _call(dtype=7) == -2
+    assert _call(variant=9) == -7
+    assert _call(variant=-1) == -7
+
+
+def test_empty_problems_are_noops():
+    assert _call(B=0) == 0
+    assert _call(C=0) == 0
+    assert _call(B=0, k=None, v=None, y=None) == 0
+
+
+def test_null_required_pointers():
+    assert _call(k=None) == -1
+    assert _call(v=None) == -1
+    assert _call(y=None) == -1
+    assert _call(w=None) == -1
+    lib = wkv4.load()
+    assert lib.wkv4_decode_step(2, 16, P, P + 0x1000, P + 0x10000, P + 0x20000, None,
+                                P + 0x30000, None, 0) == -1
+
+
+def test_overlapping_outputs_are_rejected():
+    # y overlapping k (B*T*C*4 = 1024 bytes)
+    assert _call(y=P + 0x10000 + 512) == -3
+    # state_out overlapping v
+    assert _call(so=P + 0x20000 + 64) == -3
+    # state_out partially overlapping state_in (equal is allowed, partial is not)
+    assert _call(si=P + 0x40000, so=P + 0x40000 + 4) == -3
+    # y overlapping the state
+    assert _call(si=P + 0x40000, y=P + 0x40000 + 8) == -3
+
+
+def test_scratch_bytes_is_host_only():
+    assert wkv4.scratch_bytes(8, 1, 768, wkv4.F16) == 0
+    assert wkv4.scratch_bytes(8, 1024, 768, wkv4.F16, wkv4.KERNEL_STEP) == 0
+    n = wkv4.scratch_bytes(8, 1024, 768, wkv4.F16, wkv4.KERNEL_SCAN)
+    assert n > 0
+    # 65536 steps, 2048 channels: per tile a flag and two fp32 triples per channel
+    big = wkv4.scratch_bytes(1, 65536, 2048, wkv4.F32, wkv4.KERNEL_SCAN)
+    assert 8e6 < big < 2e7
+    with pytest.raises(wkv4.Wkv4Error):
+        wkv4.scratch_bytes(1, 8, 8, 9)
