@@ -65,7 +65,6 @@ enum {
     WKV4_ERR_ALIAS = -3,   /* y or the output state overlaps an input it must not */
     WKV4_ERR_CUDA = -4,    /* a CUDA runtime call or kernel launch failed */
     WKV4_ERR_TIMEOUT = -5, /* a bounded device-side wait ran out (see wkv4_device_error) */
-    WKV4_ERR_ALLOC = -6,   /* stream-ordered scratch allocation failed */
     WKV4_ERR_VARIANT = -7  /* unknown kernel variant */
 };
 
@@ -84,11 +83,8 @@ enum {
  *               input is WKV4_ERR_ALIAS.
  *   stream      CUDA stream of the call.
  *   dtype       WKV4_F32, WKV4_F16 or WKV4_BF16.
- * Scratch: for long T the forward needs a small stream-ordered scratch
- * buffer (per-segment summaries), taken from a library-owned CUDA memory pool
- * on `stream` and returned to it on `stream`; WKV4_ERR_ALLOC if that fails.
- * Returns WKV4_OK or an error code; a device-side wait that ran out is
- * reported by wkv4_device_error().
+ * The call allocates no memory.  Returns WKV4_OK or an error code; a
+ * device-side wait that ran out is reported by wkv4_device_error().
  */
 WKV4_API int wkv4_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
                  const void* k, const void* v, const float* state_in, void* y,
@@ -98,8 +94,8 @@ WKV4_API int wkv4_forward(int64_t B, int64_t T, int64_t C, const float* w, const
 enum {
     WKV4_KERNEL_AUTO = 0,     /* what wkv4_forward picks */
     WKV4_KERNEL_SEQ = 1,      /* channel-parallel, sequential over T, TMA-staged time tiles */
-    WKV4_KERNEL_SCAN = 2,     /* chunked scan over (channel tile x time segment), TMA loads */
-    WKV4_KERNEL_SCAN_LDG = 3, /* the chunked scan with element-wise loads (any alignment) */
+    WKV4_KERNEL_SCAN = 2,     /* chunked scan, time segments chained in a thread-block cluster */
+    WKV4_KERNEL_SCAN_LDG = 3, /* the chunked scan with element-wise loads and stores */
     WKV4_KERNEL_STEP = 4      /* exact per-step max-trick, one thread per channel (any T) */
 };
 
@@ -124,15 +120,10 @@ WKV4_API int wkv4_forward_variant(int64_t B, int64_t T, int64_t C, const float* 
 WKV4_API int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float* u, const void* k,
                      const void* v, float* state, void* y, wkv4_stream_t stream, int dtype);
 
-/* Bytes of stream-ordered scratch wkv4_forward_variant would take for this
- * shape (0 when none), written to *bytes.  Host-only, no CUDA call. */
-WKV4_API int wkv4_forward_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype, int variant,
-                               size_t* bytes);
-
 /*
- * Device-side error word of the current device (bit 0: a look-back wait ran
- * out; bit 1: a TMA completion wait ran out).  Synchronises the device, reads
- * the word, and clears it when `reset` is non-zero.  Returns WKV4_OK when the
+ * Device-side error word of the current device (bit 1: a bounded wait for a
+ * TMA copy ran out).  Synchronises the device, reads the word, and clears it
+ * when `reset` is non-zero.  Returns WKV4_OK when the
  * word is zero, WKV4_ERR_TIMEOUT when a wait ran out, WKV4_ERR_CUDA when the
  * read itself failed.
  */

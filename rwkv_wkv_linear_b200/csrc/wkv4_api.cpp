@@ -1,16 +1,13 @@
 // C ABI of the RWKV-4 WKV forward / decode step: argument checks, kernel
-// choice, TMA descriptors and stream-ordered scratch.  Every step of the
+// choice and TMA descriptors.  Every step of the
 // computation runs in the kernels of wkv4_kernels.cu; nothing here computes.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
-#include <atomic>
-#include <chrono>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
-#include <random>
 
 #include "../../include/wkv4.h"
 #include "wkv4_internal.h"
@@ -18,8 +15,6 @@
 namespace {
 
 using wkv4::FwdArgs;
-
-constexpr int kMaxDevices = 64;
 
 // ------------------------------------------------------------------ helpers
 
@@ -81,63 +76,6 @@ bool tma_eligible(const FwdArgs& a) {
            is_aligned(a.y, 16) && a.T < (1ll << 31) && a.C < (1ll << 31) && a.B < (1ll << 31);
 }
 
-// Per-call epoch that tags the scan's cross-CTA flags, so stale flags left in
-// reused scratch memory never match.  Starts at a random point.
-std::atomic<unsigned long long>& epoch_counter() {
-    static std::atomic<unsigned long long> ctr{[] {
-        std::random_device rd;
-        unsigned long long x = ((unsigned long long)rd() << 32) ^ rd() ^
-                               (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
-        return (x & ((1ull << 40) - 1)) + 1;
-    }()};
-    return ctr;
-}
-
-// Library-owned memory pool per device (release threshold: keep everything),
-// so stream-ordered scratch is recycled without returning to the driver.
-cudaMemPool_t device_pool(int dev) {
-    static cudaMemPool_t pools[kMaxDevices] = {};
-    static std::mutex mu;
-    if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lk(mu);
-    if (!pools[dev]) {
-        cudaMemPoolProps props;
-        std::memset(&props, 0, sizeof(props));
-        props.allocType = cudaMemAllocationTypePinned;
-        props.handleTypes = cudaMemHandleTypeNone;
-        props.location.type = cudaMemLocationTypeDevice;
-        props.location.id = dev;
-        cudaMemPool_t pool = nullptr;
-        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
-        unsigned long long keep = ~0ull;
-        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-        pools[dev] = pool;
-    }
-    return pools[dev];
-}
-
-int alloc_scratch(void** ptr, size_t bytes, cudaStream_t stream) {
-    *ptr = nullptr;
-    if (bytes == 0) return WKV4_OK;
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return WKV4_ERR_CUDA;
-    cudaError_t e;
-    if (cap != cudaStreamCaptureStatusNone) {
-        e = cudaMallocAsync(ptr, bytes, stream);  // becomes a graph memory node
-    } else {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return WKV4_ERR_CUDA;
-        cudaMemPool_t pool = device_pool(dev);
-        if (!pool) return WKV4_ERR_ALLOC;
-        e = cudaMallocFromPoolAsync(ptr, bytes, pool, stream);
-    }
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return WKV4_ERR_ALLOC;
-    }
-    return WKV4_OK;
-}
-
 int check_common(int64_t B, int64_t T, int64_t C, int dtype) {
     if (B < 0 || T < 0 || C < 0) return WKV4_ERR_ARG;
     if (dtype != WKV4_F32 && dtype != WKV4_F16 && dtype != WKV4_BF16) return WKV4_ERR_DTYPE;
@@ -176,18 +114,8 @@ int run_scan(const FwdArgs& a, bool want_tma) {
             !encode_btc(&ty, a.y, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t))
             return WKV4_ERR_CUDA;
     }
-    void* scratch = nullptr;
-    const size_t bytes = wkv4::scan_scratch_bytes(a.B, a.T, a.C, a.dtype);
-    int rc = alloc_scratch(&scratch, bytes, a.stream);
-    if (rc != WKV4_OK) return rc;
-    const unsigned long long epoch = epoch_counter().fetch_add(1) & ((1ull << 62) - 1);
-    rc = cuda_status(wkv4::launch_scan(a, tma ? &tk : nullptr, tma ? &tv : nullptr,
-                                       tma ? &ty : nullptr, scratch, epoch));
-    if (scratch) {
-        const int rc2 = cuda_status(cudaFreeAsync(scratch, a.stream));
-        if (rc == WKV4_OK) rc = rc2;
-    }
-    return rc;
+    return cuda_status(wkv4::launch_scan(a, tma ? &tk : nullptr, tma ? &tv : nullptr,
+                                         tma ? &ty : nullptr));
 }
 
 int run_seq(const FwdArgs& a) {
@@ -261,25 +189,6 @@ int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float* u, const
     return cuda_status(wkv4::launch_decode(a));
 }
 
-int wkv4_forward_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype, int variant,
-                               size_t* bytes) {
-    if (!bytes) return WKV4_ERR_ARG;
-    *bytes = 0;
-    int rc = check_common(B, T, C, dtype);
-    if (rc != WKV4_OK) return rc;
-    if (variant < WKV4_KERNEL_AUTO || variant > WKV4_KERNEL_STEP) return WKV4_ERR_VARIANT;
-    if (B == 0 || C == 0 || T <= 1) return WKV4_OK;
-    if (variant == WKV4_KERNEL_STEP) return WKV4_OK;
-    if (variant == WKV4_KERNEL_AUTO || variant == WKV4_KERNEL_SEQ) {
-        // same decision as the call itself for aligned pointers
-        FwdArgs a{B, T, C, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dtype, nullptr};
-        const int pick = variant == WKV4_KERNEL_SEQ ? WKV4_KERNEL_SEQ : pick_variant(a);
-        if (pick == WKV4_KERNEL_SEQ && tma_eligible(a)) return WKV4_OK;
-    }
-    *bytes = wkv4::scan_scratch_bytes(B, T, C, dtype);
-    return WKV4_OK;
-}
-
 int wkv4_device_error(int reset) {
     unsigned bits = 0;
     if (wkv4::read_device_error(&bits, reset != 0) != cudaSuccess) {
@@ -297,7 +206,6 @@ const char* wkv4_status_string(int status) {
         case WKV4_ERR_ALIAS: return "output overlaps an input";
         case WKV4_ERR_CUDA: return "CUDA runtime error";
         case WKV4_ERR_TIMEOUT: return "a bounded device-side wait ran out";
-        case WKV4_ERR_ALLOC: return "scratch allocation failed";
         case WKV4_ERR_VARIANT: return "unknown kernel variant";
         default: return "unknown status";
     }

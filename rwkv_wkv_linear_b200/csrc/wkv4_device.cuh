@@ -1,8 +1,8 @@
 // Device-side building blocks of the RWKV-4 WKV kernels (sm_100a).
 //
-// Inside the kernels the state triple is kept in log2 units: A = a 2^p,
-// D = b 2^p, and k is scaled by log2(e) on load, so every exponential is one
-// ex2.approx.  The per-channel numerator / denominator / max state in fp32
+// Inside the chunked kernels the state triple is kept in log2 units:
+// A = a 2^p, D = b 2^p, with the max p in fp64, and every exponential is one
+// ex2.approx of an fp32 difference k log2(e) - r formed by one FMA.  The per-channel numerator / denominator / max state in fp32
 // with the max-trick is the one of "RWKV in a self-built engine: a second
 // non-attention paradigm (WKV/RNN)" (Methods table, "Precision").
 //
@@ -12,7 +12,7 @@
 // summary and reuses e_i for its outputs (plus one reciprocal), instead of
 // two ex2 and a reciprocal for the per-step max-trick.  This is exact
 // algebra; it is taken only when the stretch's exponents stay well inside
-// fp32 range (kmax - kmin <= kFastRange + min(0, u), u <= kFastMaxU,
+// fp32 range (in nats: kmax - kmin <= kFastRange + min(0, u), u <= kFastMaxU,
 // w <= kFastMaxW, and a carried state at most kFastStateLift above r), so
 // every denominator is >= 2^-80 and anything that underflows is below 2^-126.
 // Otherwise the stretch falls back to the per-step max-trick.
@@ -32,23 +32,28 @@
 namespace wkv4 {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
+constexpr double kLog2eD = 1.4426950408889634;
+constexpr double kLn2D = 0.6931471805599453;
 constexpr float kEmptyMaxNat = -1e38f;               // max of the empty state (natural units)
-constexpr float kEmptyMax2 = -1e38f * 1.4426950408889634f;
-constexpr float kFastRange = 80.f;                   // log2 units
-constexpr float kFastStateLift = 64.f;               // log2 units
-constexpr float kFastMaxU = 64.f;                    // log2 units
-constexpr float kFastMaxW = 0.5f;                    // log2 units per step
+constexpr double kEmptyMax2 = -1e38 * 1.4426950408889634;
+// fixed-reference chunk path limits (natural units)
+constexpr float kFastRange = 55.f;       // max k - min k (+ min(0, u)) within a chunk
+constexpr float kFastStateLift = 44.f;   // carried state's max above the chunk's max k
+constexpr float kFastMaxU = 44.f;
+constexpr float kFastMaxW = 0.35f;
 
 // device error word bits
-constexpr unsigned kErrLookback = 1u;
 constexpr unsigned kErrTmaWait = 2u;
 
 // bounded waits: polls before a wait gives up (each poll sleeps ~100 ns or more)
 constexpr uint32_t kMaxPolls = 1u << 22;
 
+// A = a 2^p, D = b 2^p.  The max p is carried in fp64 inside the kernels, so
+// that adding n*w to a large max loses nothing; it is rounded to fp32 only at
+// the state buffers, with the rounding folded back into a and b.
 struct St {
-    float a, b, p;
+    float a, b;
+    double p;
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -62,65 +67,88 @@ __device__ __forceinline__ St empty_state() { return {0.f, 0.f, kEmptyMax2}; }
 // X followed by a stretch summarised (from the empty state) as Y, the stretch
 // spanning n steps; nw2 = n * w (log2 units).  The larger of the two scale
 // factors is exactly 1, so one ex2 serves.
-__device__ __forceinline__ St combine(St x, St y, float nw2) {
-    const float px = x.p + nw2;
-    const float d = px - y.p;
-    const float f = ex2(-fabsf(d));
-    const bool xbig = d >= 0.f;
+__device__ __forceinline__ St combine(St x, St y, double nw2) {
+    const double px = x.p + nw2;
+    const double d = px - y.p;
+    const float f = ex2((float)-fabs(d));
+    const bool xbig = d >= 0.0;
     const float fx = xbig ? 1.f : f, fy = xbig ? f : 1.f;
     return {fmaf(x.a, fx, y.a * fy), fmaf(x.b, fx, y.b * fy), xbig ? px : y.p};
 }
 
 // (A, D) at reference r with D a normal positive float -> triple with b in [1, 2),
 // by an exact power-of-two rescale.
-__device__ __forceinline__ St normalized(float A, float D, float r) {
+__device__ __forceinline__ St normalized(float A, float D, double r) {
     const int e = ((__float_as_int(D) >> 23) & 0xff) - 127;
     const float s = __int_as_float((127 - e) << 23);
-    return {A * s, D * s, r + (float)e};
+    return {A * s, D * s, r + (double)e};
 }
 
-// One exact max-trick step in log2 units on state s with input
-// (x = k log2e, v): returns the output and advances the state.
-__device__ __forceinline__ float exact_step(St& s, float x, float v, float w2, float u2) {
-    const float q = fmaxf(s.p, u2 + x);
-    const float f1 = ex2(s.p - q), f2 = ex2(u2 + x - q);
+// One exact max-trick step (log2 units, fp64 max) with input k (natural), v:
+// returns the output and advances the state.  w2, u2 = w, u in log2 units.
+__device__ __forceinline__ float exact_step(St& s, float k, float v, double w2, double u2) {
+    const double x = (double)k * kLog2eD;
+    const double q = fmax(s.p, u2 + x);
+    const float f1 = ex2((float)(s.p - q)), f2 = ex2((float)(u2 + x - q));
     const float y = __fdividef(fmaf(f1, s.a, f2 * v), fmaf(f1, s.b, f2));
-    const float q2 = fmaxf(s.p + w2, x);
-    const float g1 = ex2(s.p + w2 - q2), g2 = ex2(x - q2);
+    const double q2 = fmax(s.p + w2, x);
+    const float g1 = ex2((float)(s.p + w2 - q2)), g2 = ex2((float)(x - q2));
     s.a = fmaf(g1, s.a, g2 * v);
     s.b = fmaf(g1, s.b, g2);
     s.p = q2;
     return y;
 }
 
-// The same step with the state, k, w and u in natural units (the units of
-// the state buffers), so a state carried over many single-step calls is
-// never converted: used by the decode step and the exact per-step kernel.
-__device__ __forceinline__ float exp_nat(float x) { return ex2(x * kLog2e); }
+// State advance only (no output).
+__device__ __forceinline__ void exact_update(St& s, float k, float v, double w2) {
+    const double x = (double)k * kLog2eD;
+    const double q2 = fmax(s.p + w2, x);
+    const float g1 = ex2((float)(s.p + w2 - q2)), g2 = ex2((float)(x - q2));
+    s.a = fmaf(g1, s.a, g2 * v);
+    s.b = fmaf(g1, s.b, g2);
+    s.p = q2;
+}
 
-__device__ __forceinline__ float exact_step_nat(St& s, float k, float v, float w, float u) {
-    const float q = fmaxf(s.p, u + k);
-    const float f1 = exp_nat(s.p - q), f2 = exp_nat(u + k - q);
+// The per-step max-trick with the state in natural units (the units of the
+// state buffers), fp64 max and accurate exp2f: the decode step and the
+// per-step kernel, where one step's rounding is carried to the next call.
+__device__ __forceinline__ float step_nat(St& s, float k, float v, float w, float u) {
+    const double kd = k;
+    const double q = fmax(s.p, (double)u + kd);
+    const float f1 = exp2f((float)(s.p - q) * kLog2e);
+    const float f2 = exp2f((float)((double)u + kd - q) * kLog2e);
     const float y = __fdividef(fmaf(f1, s.a, f2 * v), fmaf(f1, s.b, f2));
-    const float q2 = fmaxf(s.p + w, k);
-    const float g1 = exp_nat(s.p + w - q2), g2 = exp_nat(k - q2);
+    const double q2 = fmax(s.p + (double)w, kd);
+    const float g1 = exp2f((float)(s.p + (double)w - q2) * kLog2e);
+    const float g2 = exp2f((float)(kd - q2) * kLog2e);
     s.a = fmaf(g1, s.a, g2 * v);
     s.b = fmaf(g1, s.b, g2);
     s.p = q2;
     return y;
 }
 
-// State advance only (no output), exact max-trick, log2 units.
-__device__ __forceinline__ void exact_update(St& s, float x, float v, float w2) {
-    const float q2 = fmaxf(s.p + w2, x);
-    const float g1 = ex2(s.p + w2 - q2), g2 = ex2(x - q2);
-    s.a = fmaf(g1, s.a, g2 * v);
-    s.b = fmaf(g1, s.b, g2);
-    s.p = q2;
+__device__ __forceinline__ bool fast_ok(float kmax, float kmin, float u, float w) {
+    return (kmax - kmin <= kFastRange + fminf(0.f, u)) && (u <= kFastMaxU) && (w <= kFastMaxW);
 }
 
-__device__ __forceinline__ bool fast_ok(float kmax, float kmin, float u2, float w2) {
-    return (kmax - kmin <= kFastRange + fminf(0.f, u2)) && (u2 <= kFastMaxU) && (w2 <= kFastMaxW);
+// fp32 state buffers <-> kernel state.  On the way out the max is rounded to
+// fp32 and the rounding error d (natural units, |d| <= half an ulp of the
+// max) is folded into a and b as a(1 + d), b(1 + d) -- e^d to first order.
+__device__ __forceinline__ St load_state_log2(const float* __restrict__ s, int64_t BC, int64_t ch) {
+    return {s[ch], s[BC + ch], (double)s[2 * BC + ch] * kLog2eD};
+}
+
+__device__ __forceinline__ void store_state_nat_d(float* __restrict__ s, int64_t BC, int64_t ch,
+                                                  float a, float b, double p_nat) {
+    const float pf = (float)p_nat;
+    const float d = (float)(p_nat - (double)pf);
+    s[ch] = fmaf(a, d, a);
+    s[BC + ch] = fmaf(b, d, b);
+    s[2 * BC + ch] = pf;
+}
+
+__device__ __forceinline__ void store_state_log2(float* __restrict__ s, int64_t BC, int64_t ch, St x) {
+    store_state_nat_d(s, BC, ch, x.a, x.b, x.p * kLn2D);
 }
 
 // ---------------------------------------------------------------- I/O dtypes

@@ -34,13 +34,9 @@ Geom scan_geom(int dtype);
 Geom seq_geom(int dtype);
 size_t dtype_size(int dtype);
 
-// Scratch of the chunked scan: per (channel tile, time segment) a flag word
-// and two fp32 triples per channel (segment aggregate, inclusive prefix).
-size_t scan_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype);
-
-// Launchers.  Tensor maps are NULL for the element-wise (LDG) variants.
+// Launchers.  Tensor maps are NULL for the element-wise (LDG) variant.
 cudaError_t launch_scan(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
-                        const CUtensorMap* ty, void* scratch, unsigned long long epoch);
+                        const CUtensorMap* ty);
 cudaError_t launch_seq(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv);
 cudaError_t launch_step(const FwdArgs& a);     // exact per-step kernel, any T >= 1
 cudaError_t launch_decode(const FwdArgs& a);   // T == 1, vectorised when aligned

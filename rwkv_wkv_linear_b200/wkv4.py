@@ -21,13 +21,12 @@ F32, F16, BF16 = 0, 1, 2
 KERNEL_AUTO, KERNEL_SEQ, KERNEL_SCAN, KERNEL_SCAN_LDG, KERNEL_STEP = 0, 1, 2, 3, 4
 
 STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_DTYPE", -3: "ERR_ALIAS", -4: "ERR_CUDA",
-          -5: "ERR_TIMEOUT", -6: "ERR_ALLOC", -7: "ERR_VARIANT"}
+          -5: "ERR_TIMEOUT", -7: "ERR_VARIANT"}
 
 _DTYPES = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
 
-EXPORTS = ("wkv4_forward", "wkv4_forward_variant", "wkv4_decode_step",
-           "wkv4_forward_scratch_bytes", "wkv4_device_error", "wkv4_status_string",
-           "wkv4_version")
+EXPORTS = ("wkv4_forward", "wkv4_forward_variant", "wkv4_decode_step", "wkv4_device_error",
+           "wkv4_status_string", "wkv4_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -56,9 +55,6 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.wkv4_forward_variant.restype = i32
             lib.wkv4_decode_step.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp, vp, i32]
             lib.wkv4_decode_step.restype = i32
-            lib.wkv4_forward_scratch_bytes.argtypes = [i64, i64, i64, i32, i32,
-                                                       ctypes.POINTER(ctypes.c_size_t)]
-            lib.wkv4_forward_scratch_bytes.restype = i32
             lib.wkv4_device_error.argtypes = [i32]
             lib.wkv4_device_error.restype = i32
             lib.wkv4_status_string.argtypes = [i32]
@@ -161,14 +157,6 @@ def decode_step(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tens
     if rc != 0:
         raise Wkv4Error(rc, "wkv4_decode_step")
     return y
-
-
-def scratch_bytes(B: int, T: int, C: int, dtype: int, variant: int = KERNEL_AUTO) -> int:
-    n = ctypes.c_size_t(0)
-    rc = load().wkv4_forward_scratch_bytes(B, T, C, dtype, variant, ctypes.byref(n))
-    if rc != 0:
-        raise Wkv4Error(rc, "wkv4_forward_scratch_bytes")
-    return int(n.value)
 
 
 def device_error(reset: bool = True) -> int:

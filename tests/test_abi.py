@@ -81,15 +81,3 @@ def test_overlapping_outputs_are_rejected():
     assert _call(si=P + 0x40000, so=P + 0x40000 + 4) == -3
     # y overlapping the state
     assert _call(si=P + 0x40000, y=P + 0x40000 + 8) == -3
-
-
-def test_scratch_bytes_is_host_only():
-    assert wkv4.scratch_bytes(8, 1, 768, wkv4.F16) == 0
-    assert wkv4.scratch_bytes(8, 1024, 768, wkv4.F16, wkv4.KERNEL_STEP) == 0
-    n = wkv4.scratch_bytes(8, 1024, 768, wkv4.F16, wkv4.KERNEL_SCAN)
-    assert n > 0
-    # 65536 steps, 2048 channels: per tile a flag and two fp32 triples per channel
-    big = wkv4.scratch_bytes(1, 65536, 2048, wkv4.F32, wkv4.KERNEL_SCAN)
-    assert 8e6 < big < 2e7
-    with pytest.raises(wkv4.Wkv4Error):
-        wkv4.scratch_bytes(1, 8, 8, 9)

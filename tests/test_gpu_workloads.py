@@ -67,7 +67,7 @@ def test_long_t65536_single_and_chained(cuda_device):
         yc[:, sl] = yi
     torch.cuda.synchronize()
     parity.check_y(yc.cpu(), y_ref, x["v"], "f32", "long chained y")
-    parity.check_state(st.cpu(), s_ref, x["v"], None, what="long chained state")
+    parity.check_state(st.cpu(), s_ref, x["v"], None, calls=16, what="long chained state")
     parity.check_y(yc.cpu(), y.cpu().double().numpy(), x["v"], "f32", "chained vs single")
 
 
@@ -90,7 +90,8 @@ def test_decode_b256_1024_steps(cuda_device):
         if y_ref is not None:
             parity.check_y(yc, y_ref, v, "bf16", f"decode step {step} y")
     torch.cuda.synchronize()
-    parity.check_state(state.cpu(), ref_state, np.array([vmax]), None, what="decode final state")
+    parity.check_state(state.cpu(), ref_state, np.array([vmax]), None, calls=wl.steps,
+                       what="decode final state")
     # one more step compared on the sampled channels only
     k, v = synth.decode_step_inputs(wl, wl.steps)
     y = wkv4.decode_step(k.to(cuda_device), v.to(cuda_device), gw, gu, state)
