@@ -15,8 +15,15 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libwkv4.so")
 SOURCES = [os.path.join(CSRC, "wkv4_kernels.cu"), os.path.join(CSRC, "wkv4_api.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("wkv4_device.cuh", "wkv4_internal.h")] + [
-    os.path.join(INCLUDE, "wkv4.h")]
+
+
+def deps():
+    """Every source the library is built from: all of csrc/ and include/."""
+    out = []
+    for d in (CSRC, INCLUDE):
+        out += [os.path.join(d, f) for f in sorted(os.listdir(d))
+                if f.endswith((".cu", ".cuh", ".cpp", ".h"))]
+    return out
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -35,7 +42,7 @@ def stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(d) > t for d in DEPS)
+    return any(os.path.getmtime(d) > t for d in deps())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

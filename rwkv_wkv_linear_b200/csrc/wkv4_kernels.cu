@@ -36,14 +36,14 @@ __device__ unsigned int g_device_error = 0;
 
 namespace wkv4 {
 
-// Kernel configurations: <IO, V, L, NW> for the scan (tile 32V channels x
-// L*NW steps), <IO, V, L, NW, NS> for the sequential kernel.
-#define WKV4_SCAN_F32 float, 1, 32, 4
-#define WKV4_SCAN_F16 __half, 2, 16, 8
-#define WKV4_SCAN_BF16 __nv_bfloat16, 2, 16, 8
-#define WKV4_SEQ_F32 float, 1, 16, 4, 4
-#define WKV4_SEQ_F16 __half, 2, 16, 4, 4
-#define WKV4_SEQ_BF16 __nv_bfloat16, 2, 16, 4, 4
+// Kernel configurations: chunk length L per dtype for the scan (a warp's
+// rows are L steps x 64 channels); <IO, L, NW, NS> for the sequential kernel
+// (64*NW channels, NS stages of L steps).
+constexpr int kScanL16 = 32;  // 16-bit I/O
+constexpr int kScanL32 = 16;  // fp32 I/O
+#define WKV4_SEQ_F32 float, 16, 2, 4
+#define WKV4_SEQ_F16 __half, 16, 4, 4
+#define WKV4_SEQ_BF16 __nv_bfloat16, 16, 4, 4
 
 size_t dtype_size(int dtype) { return dtype == WKV4_F32 ? 4 : 2; }
 
@@ -64,43 +64,16 @@ static cudaError_t ensure_smem_attr(DeviceFlags& f, Kern kern, size_t smem) {
     return e;
 }
 
-template <typename IO, int V, int L, int NW>
-static Geom scan_geom_t() {
-    using Sh = ScanShape<IO, V, L, NW, 1>;
-    return {Sh::kCg, L, Sh::kThreads, Sh::kSmem};
-}
-template <typename IO, int V, int L, int NW, int NS>
+template <typename IO, int L, int NW, int NS>
 static Geom seq_geom_t() {
-    using Sh = SeqShape<IO, V, L, NW, NS>;
+    using Sh = SeqShape<IO, L, NW, NS>;
     return {Sh::kCw, L, Sh::kThreads, Sh::kSmem};
 }
 
-// Alternative fp16 tile shapes, selected with WKV4_SCAN_CFG=1..3 (tuning).
-#define WKV4_SCAN_F16_1 __half, 1, 16, 8
-#define WKV4_SCAN_F16_2 __half, 1, 32, 4
-#define WKV4_SCAN_F16_3 __half, 2, 8, 8
-
-static int scan_cfg() {
-    static const int cfg = [] {
-        const char* env = std::getenv("WKV4_SCAN_CFG");
-        const int v = env ? std::atoi(env) : 0;
-        return (v >= 0 && v <= 3) ? v : 0;
-    }();
-    return cfg;
-}
-
-// TMA boxes: scan boxes are one warp's rows (box_t = L); seq boxes one stage.
+// TMA boxes: a scan box is one warp's rows (64 channels x L steps).
 Geom scan_geom(int dtype) {
-    if (dtype == WKV4_F32) return scan_geom_t<WKV4_SCAN_F32>();
-    if (dtype == WKV4_F16) {
-        switch (scan_cfg()) {
-            case 1: return scan_geom_t<WKV4_SCAN_F16_1>();
-            case 2: return scan_geom_t<WKV4_SCAN_F16_2>();
-            case 3: return scan_geom_t<WKV4_SCAN_F16_3>();
-            default: return scan_geom_t<WKV4_SCAN_F16>();
-        }
-    }
-    return scan_geom_t<WKV4_SCAN_BF16>();
+    const int L = dtype == WKV4_F32 ? kScanL32 : kScanL16;
+    return {64, L, 0, 0};
 }
 
 Geom seq_geom(int dtype) {
@@ -115,38 +88,107 @@ static int sm_count() {
     return n;
 }
 
-// Cluster size: the largest power of two <= min(8, segments) whose grid
-// (tiles x cluster size) still fits in one wave of resident CTAs; at least 1.
-// WKV4_SCAN_CLUSTER=1|2|4|8 overrides (tuning).
-static int pick_cluster(int64_t tiles, int64_t nseg, int blocks_per_sm) {
-    const char* env = std::getenv("WKV4_SCAN_CLUSTER");
-    if (env) {
-        const int v = std::atoi(env);
-        if (v == 1 || v == 2 || v == 4 || v == 8) return v;
-    }
-    const int64_t cap = (int64_t)blocks_per_sm * sm_count();
-    int nc = 1;
-    while (nc < 8 && nc * 2 <= nseg && tiles * nc * 2 <= cap) nc *= 2;
-    return nc;
+static int env_int(const char* name, int dflt) {
+    const char* e = std::getenv(name);
+    return e ? std::atoi(e) : dflt;
 }
 
-template <typename IO, int V, int L, int NW, int NB, bool kTMA>
-static cudaError_t launch_scan_nb(const FwdArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                                  const CUtensorMap& ty, ScanParams p, int nc, int64_t tiles) {
-    using Sh = ScanShape<IO, V, L, NW, NB>;
-    auto kern = wkv4_scan_kernel<IO, V, L, NW, NB, kTMA>;
+constexpr size_t kMaxSmem = 227 * 1024;
+constexpr int kNwChoices[3] = {4, 8, 16};
+
+// Resident CTAs per SM of one scan instantiation for each warp count, cached
+// per device (0 = that warp count does not fit).
+struct ScanOcc {
+    std::atomic<int> bps[64][3];
+};
+
+template <typename IO, int L, int NB, bool kTMA>
+static cudaError_t scan_occupancy(int (&bps)[3]) {
     static DeviceFlags attr;
-    cudaError_t e = ensure_smem_attr(attr, kern, Sh::kSmem);
+    static ScanOcc occ;
+    auto kern = wkv4_scan_kernel<IO, L, NB, kTMA>;
+    cudaError_t e = ensure_smem_attr(attr, kern, kMaxSmem);
     if (e != cudaSuccess) return e;
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    for (int i = 0; i < 3; ++i) {
+        const ScanLayout<IO, L, NB> lay{kNwChoices[i]};
+        int v = (dev >= 0 && dev < 64) ? occ.bps[dev][i].load(std::memory_order_relaxed) : 0;
+        if (v == 0) {
+            v = -1;
+            if (lay.bytes() <= kMaxSmem) {
+                int n = 0;
+                if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * kNwChoices[i],
+                                                                       lay.bytes())) != cudaSuccess)
+                    return e;
+                v = n > 0 ? n : -1;
+            }
+            if (dev >= 0 && dev < 64) occ.bps[dev][i].store(v, std::memory_order_relaxed);
+        }
+        bps[i] = v > 0 ? v : 0;
+    }
+    return cudaSuccess;
+}
+
+// Launch shape of the scan: warps per CTA (NW) and cluster size (NC).
+// Preference: the fewest (waves x rounds), where a wave is the CTAs the GPU
+// holds at once and a round is one pass of the cluster over NC segments;
+// then the larger grid.  WKV4_SCAN_NW / WKV4_SCAN_CLUSTER override (tuning).
+struct ScanShape {
+    int nw, nc, rounds, nb;
+};
+
+template <typename IO, int L, bool kTMA>
+static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
+    int b1[3], b2[3];
+    cudaError_t e = scan_occupancy<IO, L, 1, kTMA>(b1);
+    if (e != cudaSuccess) return e;
+    if ((e = scan_occupancy<IO, L, 2, kTMA>(b2)) != cudaSuccess) return e;
+    const int sms = sm_count();
+    const int force_nw = env_int("WKV4_SCAN_NW", 0), force_nc = env_int("WKV4_SCAN_CLUSTER", 0);
+    bool have = false;
+    int64_t best_cost = 0, best_grid = 0;
+    for (int i = 0; i < 3; ++i) {
+        const int nw = kNwChoices[i];
+        if (force_nw && nw != force_nw) continue;
+        const int64_t nseg = (T + (int64_t)nw * L - 1) / ((int64_t)nw * L);
+        for (int nc = 1; nc <= kMaxCluster; nc *= 2) {
+            if (force_nc ? nc != force_nc : (nc > 1 && nc > nseg)) continue;
+            const int64_t rounds = (nseg + nc - 1) / nc;
+            const int nb = rounds > 1 ? 2 : 1;
+            const int bps = nb == 1 ? b1[i] : b2[i];
+            if (bps <= 0) continue;
+            const int64_t cap = (int64_t)bps * sms / nc * nc;  // whole clusters
+            if (cap <= 0) continue;
+            const int64_t grid = tiles * nc;
+            const int64_t waves = (grid + cap - 1) / cap;
+            const int64_t cost = waves * rounds;
+            if (!have || cost < best_cost || (cost == best_cost && grid > best_grid)) {
+                have = true;
+                best_cost = cost;
+                best_grid = grid;
+                out = {nw, nc, (int)rounds, nb};
+            }
+        }
+    }
+    return have ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+template <typename IO, int L, int NB, bool kTMA>
+static cudaError_t launch_scan_nb(const FwdArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const CUtensorMap& ty, const ScanParams& p, const ScanShape& sh,
+                                  int64_t tiles) {
+    auto kern = wkv4_scan_kernel<IO, L, NB, kTMA>;
+    const ScanLayout<IO, L, NB> lay{sh.nw};
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)(tiles * nc), 1, 1);
-    cfg.blockDim = dim3(Sh::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = Sh::kSmem;
+    cfg.gridDim = dim3((unsigned)(tiles * sh.nc), 1, 1);
+    cfg.blockDim = dim3(32 * sh.nw, 1, 1);
+    cfg.dynamicSmemBytes = lay.bytes();
     cfg.stream = a.stream;
     cudaLaunchAttribute attrs[1];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
-    attrs[0].val.clusterDim.x = (unsigned)nc;
+    attrs[0].val.clusterDim.x = (unsigned)sh.nc;
     attrs[0].val.clusterDim.y = 1;
     attrs[0].val.clusterDim.z = 1;
     cfg.attrs = attrs;
@@ -154,14 +196,13 @@ static cudaError_t launch_scan_nb(const FwdArgs& a, const CUtensorMap& tk, const
     return cudaLaunchKernelEx(&cfg, kern, tk, tv, ty, p);
 }
 
-template <typename IO, int V, int L, int NW, bool kTMA>
+template <typename IO, int L, bool kTMA>
 static cudaError_t launch_scan_t(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
                                  const CUtensorMap* ty) {
-    using Sh1 = ScanShape<IO, V, L, NW, 1>;
-    ScanParams p;
+    ScanParams p{};
     p.T = a.T;
     p.C = a.C;
-    p.CGB = (int)((a.C + Sh1::kCg - 1) / Sh1::kCg);
+    p.CGB = (int)((a.C + 63) / 64);
     p.w = a.w;
     p.u = a.u;
     p.k = a.k;
@@ -170,33 +211,20 @@ static cudaError_t launch_scan_t(const FwdArgs& a, const CUtensorMap* tk, const 
     p.y = a.y;
     p.state_out = a.state_out;
     p.BC = a.B * a.C;
+    p.bulk_params = ((uintptr_t)a.w % 16 == 0) && ((uintptr_t)a.u % 16 == 0) &&
+                    ((uintptr_t)a.state_in % 16 == 0) && (a.C % 4 == 0);
     const int64_t tiles = a.B * p.CGB;
-    const int64_t nseg = (a.T + Sh1::kTs - 1) / Sh1::kTs;
-    // resident CTAs per SM of the single-buffer kernel, cached per device
-    auto k1 = wkv4_scan_kernel<IO, V, L, NW, 1, kTMA>;
-    static DeviceFlags attr1;
-    static std::atomic<int> bps_cache[64];
-    cudaError_t e = ensure_smem_attr(attr1, k1, Sh1::kSmem);
+    ScanShape sh;
+    cudaError_t e = pick_scan_shape<IO, L, kTMA>(tiles, a.T, sh);
     if (e != cudaSuccess) return e;
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    int bps = (dev >= 0 && dev < 64) ? bps_cache[dev].load(std::memory_order_relaxed) : 0;
-    if (bps <= 0) {
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k1, Sh1::kThreads,
-                                                               Sh1::kSmem)) != cudaSuccess)
-            return e;
-        bps = bps > 0 ? bps : 1;
-        if (dev >= 0 && dev < 64) bps_cache[dev].store(bps, std::memory_order_relaxed);
-    }
-    const int nc = pick_cluster(tiles, nseg, bps);
-    p.rounds = (int)((nseg + nc - 1) / nc);
+    p.rounds = sh.rounds;
     CUtensorMap dummy;
     std::memset(&dummy, 0, sizeof(dummy));
     const CUtensorMap& mk = tk ? *tk : dummy;
     const CUtensorMap& mv = tv ? *tv : dummy;
     const CUtensorMap& my = ty ? *ty : dummy;
-    if (p.rounds == 1) return launch_scan_nb<IO, V, L, NW, 1, kTMA>(a, mk, mv, my, p, nc, tiles);
-    return launch_scan_nb<IO, V, L, NW, 2, kTMA>(a, mk, mv, my, p, nc, tiles);
+    if (sh.nb == 1) return launch_scan_nb<IO, L, 1, kTMA>(a, mk, mv, my, p, sh, tiles);
+    return launch_scan_nb<IO, L, 2, kTMA>(a, mk, mv, my, p, sh, tiles);
 }
 
 cudaError_t launch_scan(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
@@ -204,30 +232,25 @@ cudaError_t launch_scan(const FwdArgs& a, const CUtensorMap* tk, const CUtensorM
     const bool tma = tk != nullptr;
     switch (a.dtype) {
         case WKV4_F32:
-            return tma ? launch_scan_t<WKV4_SCAN_F32, true>(a, tk, tv, ty)
-                       : launch_scan_t<WKV4_SCAN_F32, false>(a, tk, tv, ty);
+            return tma ? launch_scan_t<float, kScanL32, true>(a, tk, tv, ty)
+                       : launch_scan_t<float, kScanL32, false>(a, tk, tv, ty);
         case WKV4_F16:
-            if (!tma) return launch_scan_t<WKV4_SCAN_F16, false>(a, tk, tv, ty);
-            switch (scan_cfg()) {
-                case 1: return launch_scan_t<WKV4_SCAN_F16_1, true>(a, tk, tv, ty);
-                case 2: return launch_scan_t<WKV4_SCAN_F16_2, true>(a, tk, tv, ty);
-                case 3: return launch_scan_t<WKV4_SCAN_F16_3, true>(a, tk, tv, ty);
-                default: return launch_scan_t<WKV4_SCAN_F16, true>(a, tk, tv, ty);
-            }
+            return tma ? launch_scan_t<__half, kScanL16, true>(a, tk, tv, ty)
+                       : launch_scan_t<__half, kScanL16, false>(a, tk, tv, ty);
         default:
-            return tma ? launch_scan_t<WKV4_SCAN_BF16, true>(a, tk, tv, ty)
-                       : launch_scan_t<WKV4_SCAN_BF16, false>(a, tk, tv, ty);
+            return tma ? launch_scan_t<__nv_bfloat16, kScanL16, true>(a, tk, tv, ty)
+                       : launch_scan_t<__nv_bfloat16, kScanL16, false>(a, tk, tv, ty);
     }
 }
 
-template <typename IO, int V, int L, int NW, int NS>
+template <typename IO, int L, int NW, int NS>
 static cudaError_t launch_seq_t(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv) {
-    using Sh = SeqShape<IO, V, L, NW, NS>;
-    auto kern = wkv4_seq_kernel<IO, V, L, NW, NS>;
+    using Sh = SeqShape<IO, L, NW, NS>;
+    auto kern = wkv4_seq_kernel<IO, L, NW, NS>;
     static DeviceFlags attr;
     cudaError_t e = ensure_smem_attr(attr, kern, Sh::kSmem);
     if (e != cudaSuccess) return e;
-    SeqParams p;
+    SeqParams p{};
     p.T = a.T;
     p.C = a.C;
     p.CGB = (int)((a.C + Sh::kCw - 1) / Sh::kCw);
@@ -251,7 +274,7 @@ cudaError_t launch_seq(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMa
 }
 
 static StepParams step_params(const FwdArgs& a) {
-    StepParams p;
+    StepParams p{};
     p.B = a.B;
     p.T = a.T;
     p.C = a.C;

@@ -1,23 +1,26 @@
 // Chunked scan over (channel tile x time segment) tiles, chained through a
 // thread-block cluster.
 //
-// A cluster of NC CTAs owns one channel tile (Cg = 32 V channels of one batch
-// row) and walks T in rounds of NC segments of Ts = NW L steps; CTA rank r
-// takes segment round * NC + r.  Inside a CTA each warp owns one chunk of L
-// steps (its rows arrive by their own TMA box and mbarrier, so a warp starts
-// as soon as its rows land) and each lane V channels.  Per round:
+// A cluster of NC CTAs owns one channel tile (Cg = 64 channels of one batch
+// row, one channel pair per lane) and walks T in rounds of NC segments of
+// Ts = NW L steps; CTA rank r takes segment round * NC + r.  NW (warps per
+// CTA) and NC are chosen at launch so that, where the GPU can hold it, the
+// whole T is one round of one wave.  Inside a CTA each warp owns one chunk of
+// L steps; its rows arrive by their own TMA box and mbarrier, so a warp
+// starts as soon as its rows land.  Per round:
 //   1. every warp summarises its chunk from the empty state (chunk_phase1);
-//   2. the chunk summaries are combined inside the CTA into the segment's
-//      aggregate, published in the CTA's shared memory;
-//   3. one cluster barrier; every warp then reads the NC aggregates of the
-//      round from its peers' shared memory (DSMEM) and folds them, from the
-//      state carried into the round, into the state at its own chunk start
-//      and the state carried into the next round;
+//   2. warp 0 scans the NW chunk summaries (the state contribution before
+//      each chunk, the segment's aggregate) and publishes the aggregate in
+//      its CTA's shared memory;
+//   3. one cluster barrier; the warps copy the NC aggregates of the round from
+//      the cluster's shared memory (DSMEM loads, all in flight together) and
+//      warp 0 folds them, from the state carried into the round, into the
+//      state at the segment start and the state carried into the next round;
 //   4. every warp emits its chunk's outputs (chunk_phase3) into its k rows
 //      and sends them out with its own TMA store.
-// The next round's tiles are prefetched into the second buffer (NB = 2).
-// There is no global scratch and no spin-wait on another CTA: all exchange is
-// through cluster shared memory and hardware cluster barriers.
+// With several rounds the next round's rows are prefetched into a second
+// buffer (NB = 2).  There is no global scratch and no spin-wait on another
+// CTA: all exchange is through cluster shared memory and hardware barriers.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -28,26 +31,38 @@ namespace wkv4 {
 
 namespace cg = cooperative_groups;
 
-template <typename IO, int V, int L, int NW, int NB>
-struct ScanShape {
-    static constexpr int kCg = 32 * V;   // channels per tile
-    static constexpr int kTs = L * NW;   // steps per segment
-    static constexpr int kThreads = 32 * NW;
+constexpr int kMaxCluster = 8;
+
+// Register cap of the scan kernel: enough CTAs per SM for the whole grid of
+// the common shapes to be resident at once.
+#ifndef WKV4_SCAN_MAXNREG
+#define WKV4_SCAN_MAXNREG 96
+#endif
+
+// Shared-memory layout for nw warps (offsets from a 1024-byte aligned base).
+template <typename IO, int L, int NB>
+struct ScanLayout {
+    static constexpr int kCg = 64;  // channels per tile: 32 lanes x 2
     static constexpr int kChunkBytes = L * kCg * (int)sizeof(IO);  // one warp's rows, one tensor
-    static constexpr int kTileBytes = NW * kChunkBytes;
-    static constexpr size_t kOffSum = (size_t)NB * 2 * kTileBytes;
-    static constexpr size_t kOffAgg = kOffSum + (size_t)NW * kCg * 16;   // a, b f32 + p f64
-    static constexpr size_t kOffBar = kOffAgg + (size_t)2 * kCg * 16;
-    static constexpr size_t kSmem = 1024 + kOffBar + (size_t)NB * NW * 8;
-    static_assert(kCg <= 256 && L <= 256, "TMA box dims");
-    static_assert((kCg * sizeof(IO)) % 16 == 0, "TMA inner box bytes");
+    static_assert(L <= 256, "TMA box dims");
     static_assert(kChunkBytes % 128 == 0, "TMA destination alignment");
+    int nw;
+    __host__ __device__ size_t tile() const { return (size_t)nw * kChunkBytes; }
+    __host__ __device__ size_t k(int buf) const { return (size_t)buf * 2 * tile(); }
+    __host__ __device__ size_t v(int buf) const { return k(buf) + tile(); }
+    __host__ __device__ size_t sums() const { return (size_t)NB * 2 * tile(); }       // [nw][Cg] x 16 B
+    __host__ __device__ size_t agg() const { return sums() + (size_t)nw * kCg * 16; }  // [2][Cg] x 16 B
+    __host__ __device__ size_t start() const { return agg() + (size_t)2 * kCg * 16; }  // [Cg] x 16 B
+    __host__ __device__ size_t peers() const { return start() + (size_t)kCg * 16; }    // [8][Cg] x 16 B
+    __host__ __device__ size_t params() const { return peers() + (size_t)8 * kCg * 16; } // w, u, state [5][Cg] f32
+    __host__ __device__ size_t bars() const { return params() + (size_t)5 * kCg * 4; }  // [NB][nw] + 1 x 8 B
+    __host__ __device__ size_t bytes() const { return 1024 + bars() + (size_t)(NB * nw + 1) * 8; }
 };
 
 struct ScanParams {
     int64_t T, C;
     int CGB;     // channel tiles per batch row
-    int rounds;  // ceil(nseg / NC)
+    int rounds;  // ceil(segments / NC)
     const float* w;
     const float* u;
     const void* k;  // element-wise variant only
@@ -56,23 +71,43 @@ struct ScanParams {
     void* y;
     float* state_out;
     int64_t BC;
+    int bulk_params;  // w, u, state_in are 16-byte aligned: fetch them by bulk copy
 };
 
-template <typename IO, int V, int L, int NW, int NB, bool kTMA>
-__global__ void __launch_bounds__(32 * NW)
+// (a, b, p) triples in shared memory, stored as three planes of n entries.
+struct TripleRef {
+    float* a;
+    float* b;
+    double* p;
+    __device__ __forceinline__ St get(int i) const { return {a[i], b[i], p[i]}; }
+    __device__ __forceinline__ void put(int i, St s) const {
+        a[i] = s.a;
+        b[i] = s.b;
+        p[i] = s.p;
+    }
+};
+
+__device__ __forceinline__ TripleRef triples(unsigned char* at, int n) {
+    float* a = reinterpret_cast<float*>(at);
+    float* b = a + n;
+    return {a, b, reinterpret_cast<double*>(b + n)};
+}
+
+template <typename IO, int L, int NB, bool kTMA>
+__global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     wkv4_scan_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __grid_constant__ CUtensorMap tmy, const ScanParams p) {
-    using Sh = ScanShape<IO, V, L, NW, NB>;
-    constexpr int Cg = Sh::kCg, Ts = Sh::kTs;
+    constexpr int Cg = ScanLayout<IO, L, NB>::kCg;
+    constexpr int kChunkBytes = ScanLayout<IO, L, NB>::kChunkBytes;
+    const int NW = blockDim.x >> 5;
+    const ScanLayout<IO, L, NB> lay{NW};
+    const int Ts = NW * L;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float* sum_a = reinterpret_cast<float*>(base + Sh::kOffSum);  // [NW][Cg]
-    float* sum_b = sum_a + NW * Cg;
-    double* sum_p = reinterpret_cast<double*>(sum_b + NW * Cg);
-    float* agg_a = reinterpret_cast<float*>(base + Sh::kOffAgg);  // [2][Cg]
-    float* agg_b = agg_a + 2 * Cg;
-    double* agg_p = reinterpret_cast<double*>(agg_b + 2 * Cg);
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(base + Sh::kOffBar);  // [NB][NW]
+    // align by offsetting the shared array itself (a round trip through an
+    // integer would lose the address space and turn every access generic)
+    unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const TripleRef sums = triples(base + lay.sums(), NW * Cg);      // [NW][Cg]
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // [NB][NW]
 
     cg::cluster_group cluster = cg::this_cluster();
     const int NC = (int)cluster.num_blocks();
@@ -82,30 +117,61 @@ __global__ void __launch_bounds__(32 * NW)
     const int64_t c0 = (int64_t)(g - b * p.CGB) * Cg;
     const int64_t T = p.T, C = p.C;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int col = lane * V;
+    const int col = lane * 2;
     const int64_t seg_stride = (int64_t)NC * Ts;  // steps per round
 
-    auto tile_k = [&](int buf) { return reinterpret_cast<IO*>(base + (size_t)buf * 2 * Sh::kTileBytes); };
-    auto tile_v = [&](int buf) {
-        return reinterpret_cast<IO*>(base + (size_t)buf * 2 * Sh::kTileBytes + Sh::kTileBytes);
-    };
-    // steps of this warp's chunk in round j
-    auto chunk_n = [&](int j) -> int {
-        const int64_t tc = (int64_t)j * seg_stride + (int64_t)rank * Ts + (int64_t)warp * L;
+    auto chunk_len = [&](int j, int q) -> int {  // steps of chunk q of this CTA in round j
+        const int64_t tc = (int64_t)j * seg_stride + (int64_t)rank * Ts + (int64_t)q * L;
         return (int)max((int64_t)0, min((int64_t)L, T - tc));
     };
-    auto issue_loads = [&](int j) {  // lane 0 of each warp, own rows of round j
-        const int buf = j % NB;
-        if (chunk_n(j) <= 0) return;
-        const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
-        uint64_t* bar = mbar + buf * NW + warp;
+    auto rows_k = [&](int buf) { return reinterpret_cast<IO*>(base + lay.k(buf)) + warp * L * Cg; };
+    auto rows_v = [&](int buf) { return reinterpret_cast<IO*>(base + lay.v(buf)) + warp * L * Cg; };
+    auto issue_loads = [&](int j) {  // lane 0 of each warp: this warp's rows of round j
         if constexpr (kTMA) {
-            mbar_arrive_expect_tx(bar, 2u * Sh::kChunkBytes);
-            tma_load_3d(tile_k(buf) + warp * L * Cg, &tmk, (int)c0, t, b, bar);
-            tma_load_3d(tile_v(buf) + warp * L * Cg, &tmv, (int)c0, t, b, bar);
+            if (chunk_len(j, warp) <= 0) return;
+            const int buf = j % NB;
+            const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
+            uint64_t* bar = mbar + buf * NW + warp;
+            mbar_arrive_expect_tx(bar, 2u * kChunkBytes);
+            tma_load_3d(rows_k(buf), &tmk, (int)c0, t, b, bar);
+            tma_load_3d(rows_v(buf), &tmv, (int)c0, t, b, bar);
         }
     };
 
+    // Per-channel w, u and the state for this tile: a full 64-channel slice
+    // with aligned pointers comes by bulk copy on its own mbarrier, issued
+    // before the tiles, so it does not queue behind other CTAs' tile traffic.
+    PairConsts cc;
+    St carry[2];  // warp 0: the state carried into the current round
+    uint64_t* pbar = mbar + NB * NW;
+    float* sw = reinterpret_cast<float*>(base + lay.params());  // [5][Cg]: w, u, a, b, p
+    const bool bulk = kTMA && p.bulk_params && c0 + Cg <= C;
+    if (bulk) {
+        if (threadIdx.x == 0) {
+            mbar_init(pbar, 1);
+            fence_mbar_init();
+            const uint32_t nb = Cg * 4;
+            const int64_t ch = (int64_t)b * C + c0;
+            mbar_arrive_expect_tx(pbar, (p.state_in ? 5u : 2u) * nb);
+            bulk_load(sw, p.w + c0, nb, pbar);
+            bulk_load(sw + Cg, p.u + c0, nb, pbar);
+            if (p.state_in) {
+                bulk_load(sw + 2 * Cg, p.state_in + ch, nb, pbar);
+                bulk_load(sw + 3 * Cg, p.state_in + p.BC + ch, nb, pbar);
+                bulk_load(sw + 4 * Cg, p.state_in + 2 * p.BC + ch, nb, pbar);
+            }
+        }
+    } else {
+        pair_wu(p.w, p.u, c0 + col, C, cc);
+        if (warp == 0) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int64_t c = c0 + col + j;
+                carry[j] = (p.state_in && c < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c)
+                                                 : empty_state();
+            }
+        }
+    }
     if constexpr (kTMA) {
         if (lane == 0) {
             if (warp == 0) {
@@ -119,24 +185,30 @@ __global__ void __launch_bounds__(32 * NW)
         }
         __syncwarp();
     }
-
-    ChanConsts cc[V];
-    channel_consts<V>(p.w, p.u, c0 + col, C, cc);
-    St carry[V];
+    if (bulk) {
+        __syncthreads();  // the params barrier is initialised
+        if (!mbar_wait_bounded(pbar, 0)) {
+            if (lane == 0) atomicOr(&g_device_error, kErrTmaWait);
+        }
 #pragma unroll
-    for (int j = 0; j < V; ++j) {
-        const int64_t c = c0 + col + j;
-        carry[j] = (p.state_in && c < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c)
-                                         : empty_state();
+        for (int j = 0; j < 2; ++j) {
+            cc.w[j] = sw[col + j];
+            cc.u[j] = sw[Cg + col + j];
+            if (warp == 0)
+                carry[j] = p.state_in ? St{sw[2 * Cg + col + j], sw[3 * Cg + col + j],
+                                           (double)sw[4 * Cg + col + j] * kLog2eD}
+                                      : empty_state();
+        }
     }
+    pair_derive(cc);
     bool failed = false;
 
     for (int round = 0; round < p.rounds; ++round) {
         const int buf = round % NB;
-        const int n = chunk_n(round);
+        const int n = chunk_len(round, warp);
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;  // segment start
-        IO* kr = tile_k(buf) + warp * L * Cg;
-        IO* vr = tile_v(buf) + warp * L * Cg;
+        IO* kr = rows_k(buf);
+        IO* vr = rows_v(buf);
         if constexpr (kTMA) {
             if (n > 0 && !failed &&
                 !mbar_wait_bounded(mbar + buf * NW + warp, (uint32_t)((round / NB) & 1))) {
@@ -163,105 +235,115 @@ __global__ void __launch_bounds__(32 * NW)
         }
 
         // ---- 1. chunk summaries
-        ChunkRegs<V, L> r;
-        St sum[V];
-        chunk_phase1<IO, V, L>(r, kr, vr, Cg, col, n, cc, sum);
+        PairRef ref;
+        St sum[2];
+        chunk_phase1<IO, L>(ref, kr, vr, Cg, col, n, cc, sum);
 #pragma unroll
-        for (int j = 0; j < V; ++j) {
-            sum_a[warp * Cg + col + j] = sum[j].a;
-            sum_b[warp * Cg + col + j] = sum[j].b;
-            sum_p[warp * Cg + col + j] = sum[j].p;
+        for (int j = 0; j < 2; ++j) sums.put(warp * Cg + col + j, sum[j]);
+        __syncthreads();
+
+        // ---- 2. warp 0: exclusive prefix of the chunk summaries (in place)
+        //         and the segment aggregate
+        const int slot = round & 1;
+        const TripleRef agg = triples(base + lay.agg() + (size_t)slot * Cg * 16, Cg);
+        const TripleRef start = triples(base + lay.start(), Cg);
+        if (warp == 0) {
+            St acc[2] = {empty_state(), empty_state()};
+#pragma unroll 1
+            for (int q = 0; q < NW; ++q) {
+                const double nq = (double)chunk_len(round, q);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int i = q * Cg + col + j;
+                    const St Sq = sums.get(i);
+                    sums.put(i, acc[j]);
+                    acc[j] = combine(acc[j], Sq, nq * cc.w2[j]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) agg.put(col + j, acc[j]);
+        }
+
+        // ---- 3. copy the cluster's aggregates of this round into local shared
+        //         memory (warp q reads peers q, q + NW, ...: the remote loads of
+        //         all warps are in flight together); warp 0 folds them
+        cluster.sync();
+        for (int q = warp; q < NC; q += NW) {
+            const float* ra = cluster.map_shared_rank(agg.a, q);
+            const float* rb = cluster.map_shared_rank(agg.b, q);
+            const double* rp = cluster.map_shared_rank(agg.p, q);
+            const TripleRef dst = triples(base + lay.peers() + (size_t)q * Cg * 16, Cg);
+            const float2 a2 = *reinterpret_cast<const float2*>(ra + col);
+            const float2 b2 = *reinterpret_cast<const float2*>(rb + col);
+            const double p0 = rp[col], p1 = rp[col + 1];
+            dst.put(col, {a2.x, b2.x, p0});
+            dst.put(col + 1, {a2.y, b2.y, p1});
+        }
+        __syncthreads();
+        if (warp == 0) {
+#pragma unroll 1
+            for (int q = 0; q < NC; ++q) {
+                const TripleRef src = triples(base + lay.peers() + (size_t)q * Cg * 16, Cg);
+                const int64_t sq = t0 + (int64_t)(q - rank) * Ts;
+                const double nq = (double)max((int64_t)0, min((int64_t)Ts, T - sq));
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    if (q == rank) start.put(col + j, carry[j]);
+                    carry[j] = combine(carry[j], src.get(col + j), nq * cc.w2[j]);
+                }
+            }
         }
         __syncthreads();
 
-        // ---- 2. exclusive prefix of the chunks before this warp; segment aggregate
-        St E[V];
-#pragma unroll
-        for (int j = 0; j < V; ++j) E[j] = empty_state();
-        for (int q = 0; q < warp; ++q) {
-            const int64_t tq = t0 + (int64_t)q * L;
-            const int nq = (int)max((int64_t)0, min((int64_t)L, T - tq));
-#pragma unroll
-            for (int j = 0; j < V; ++j) {
-                const St Sq = {sum_a[q * Cg + col + j], sum_b[q * Cg + col + j], sum_p[q * Cg + col + j]};
-                E[j] = combine(E[j], Sq, (double)nq * cc[j].w2);
-            }
-        }
-        const int slot = round & 1;
-        if (warp == NW - 1) {
-#pragma unroll
-            for (int j = 0; j < V; ++j) {
-                const St A = combine(E[j], sum[j], (double)n * cc[j].w2);
-                agg_a[slot * Cg + col + j] = A.a;
-                agg_b[slot * Cg + col + j] = A.b;
-                agg_p[slot * Cg + col + j] = A.p;
-            }
-        }
-
-        // ---- 3. exchange segment aggregates across the cluster
-        cluster.sync();
-        St P[V], next[V];
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            P[j] = carry[j];
-            next[j] = carry[j];
-        }
-        for (int q = 0; q < NC; ++q) {
-            const int64_t sq = t0 + (int64_t)(q - rank) * Ts;
-            const int nq = (int)max((int64_t)0, min((int64_t)Ts, T - sq));
-            const float* pa = cluster.map_shared_rank(agg_a + slot * Cg, q);
-            const float* pb = cluster.map_shared_rank(agg_b + slot * Cg, q);
-            const double* pp = cluster.map_shared_rank(agg_p + slot * Cg, q);
-#pragma unroll
-            for (int j = 0; j < V; ++j) {
-                const St Aq = {pa[col + j], pb[col + j], pp[col + j]};
-                next[j] = combine(next[j], Aq, (double)nq * cc[j].w2);
-                if (q + 1 == rank) P[j] = next[j];
-            }
-        }
-
         // ---- 4. outputs of this warp's chunk
-        St S[V];
+        St S[2];
 #pragma unroll
-        for (int j = 0; j < V; ++j) S[j] = combine(P[j], E[j], (double)(warp * L) * cc[j].w2);
+        for (int j = 0; j < 2; ++j)
+            S[j] = combine(start.get(col + j), sums.get(warp * Cg + col + j),
+                           (double)(warp * L) * cc.w2[j]);
         if constexpr (kTMA) {
-            auto out_vec = [&](int i, const float (&yv)[V]) { store_vec<IO, V>(kr + i * Cg + col, yv); };
-            auto out_one = [&](int i, int j, float yv) { kr[i * Cg + col + j] = Io<IO>::from_f(yv); };
-            chunk_phase3<IO, V, L>(r, kr, vr, Cg, col, n, S, cc, out_vec, out_one);
+            // y is staged in place of k (step i reads k_i before writing y_i)
+            auto out_pair = [=](int i, f2 y) { Pair<IO>::store(kr + i * Cg + col, y); };
+            auto out_one = [=](int i, int j, float y) { kr[i * Cg + col + j] = Io<IO>::from_f(y); };
+            chunk_phase3<IO, L>(ref, kr, vr, Cg, col, n, S, cc, out_pair, out_one);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0 && n > 0) {
-                if (!failed) tma_store_3d(&tmy, kr, (int)c0, (int)(t0 + warp * L), b);
-                bulk_commit();
-                bulk_wait_read_all();  // rows free for the next load into this buffer
-                if (round + NB < p.rounds) issue_loads(round + NB);
-            } else if (lane == 0 && round + NB < p.rounds) {
-                issue_loads(round + NB);
+            if (lane == 0) {
+                if (n > 0 && !failed) {
+                    tma_store_3d(&tmy, kr, (int)c0, (int)(t0 + warp * L), b);
+                    bulk_commit();
+                }
+                if (round + NB < p.rounds) {
+                    bulk_wait_read_all();  // rows free for the next load into this buffer
+                    issue_loads(round + NB);
+                }
             }
             __syncwarp();
         } else {
             IO* yg = static_cast<IO*>(p.y);
             const int64_t ybase = ((int64_t)b * T + t0 + warp * L) * C + c0 + col;
-            auto out_one = [&](int i, int j, float yv) {
-                if (c0 + col + j < C) yg[ybase + (int64_t)i * C + j] = Io<IO>::from_f(yv);
+            const int64_t cpair = c0 + col;
+            auto out_one = [=](int i, int j, float y) {
+                if (cpair + j < C) yg[ybase + (int64_t)i * C + j] = Io<IO>::from_f(y);
             };
-            auto out_vec = [&](int i, const float (&yv)[V]) {
-#pragma unroll
-                for (int j = 0; j < V; ++j) out_one(i, j, yv[j]);
+            auto out_pair = [=](int i, f2 y) {
+                if (cpair < C) yg[ybase + (int64_t)i * C] = Io<IO>::from_f(lo(y));
+                if (cpair + 1 < C) yg[ybase + (int64_t)i * C + 1] = Io<IO>::from_f(hi(y));
             };
-            chunk_phase3<IO, V, L>(r, kr, vr, Cg, col, n, S, cc, out_vec, out_one);
+            chunk_phase3<IO, L>(ref, kr, vr, Cg, col, n, S, cc, out_pair, out_one);
             __syncwarp();
         }
-#pragma unroll
-        for (int j = 0; j < V; ++j) carry[j] = next[j];
     }
 
     if (rank == 0 && warp == 0 && p.state_out) {
 #pragma unroll
-        for (int j = 0; j < V; ++j) {
+        for (int j = 0; j < 2; ++j) {
             const int64_t c = c0 + col + j;
             if (c < C) store_state_log2(p.state_out, p.BC, (int64_t)b * C + c, carry[j]);
         }
+    }
+    if constexpr (kTMA) {
+        if (lane == 0) bulk_wait_read_all();  // the staged rows stay valid until read
     }
     // peers may still be reading this CTA's aggregates
     cluster.sync();

@@ -1,11 +1,10 @@
 // Channel-parallel kernel, sequential over T.
 //
-// Each thread owns V channels and walks their whole sequence chunk by chunk
+// Each thread owns a channel pair and walks its whole sequence chunk by chunk
 // (chunk_phase1 -> outputs from the carried state -> carried state combined
-// with the chunk summary).  The CTA's Cw = 32 V NW channels are staged through
+// with the chunk summary).  The CTA's Cw = 64 NW channels are staged through
 // an NS-deep ring of TMA time tiles [L steps x Cw channels] with one mbarrier
-// per stage; y leaves with 128-bit-or-narrower vector stores straight from
-// registers.  Suited to shapes with many channels (B C large), where channel
+// per stage; y leaves with pair stores straight from registers.  Suited to shapes with many channels (B C large), where channel
 // parallelism alone fills the GPU and no cross-CTA exchange is needed.
 #pragma once
 
@@ -13,9 +12,9 @@
 
 namespace wkv4 {
 
-template <typename IO, int V, int L, int NW, int NS>
+template <typename IO, int L, int NW, int NS>
 struct SeqShape {
-    static constexpr int kCw = 32 * V * NW;  // channels per CTA
+    static constexpr int kCw = 64 * NW;  // channels per CTA
     static constexpr int kThreads = 32 * NW;
     static constexpr int kStageBytes = L * kCw * (int)sizeof(IO);  // one tensor, one stage
     static constexpr size_t kSmem = 1024 + 2 * (size_t)NS * kStageBytes + NS * 8;
@@ -33,14 +32,16 @@ struct SeqParams {
     int64_t BC;
 };
 
-template <typename IO, int V, int L, int NW, int NS>
+template <typename IO, int L, int NW, int NS>
 __global__ void __launch_bounds__(32 * NW)
     wkv4_seq_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                     const SeqParams p) {
-    using Sh = SeqShape<IO, V, L, NW, NS>;
+    using Sh = SeqShape<IO, L, NW, NS>;
     constexpr int Cw = Sh::kCw;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    // align by offsetting the shared array itself (a round trip through an
+    // integer would lose the address space and turn every access generic)
+    unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     IO* sk = reinterpret_cast<IO*>(base);                         // [NS][L][Cw]
     IO* sv = reinterpret_cast<IO*>(base + NS * Sh::kStageBytes);  // [NS][L][Cw]
     uint64_t* mbar = reinterpret_cast<uint64_t*>(base + 2 * NS * Sh::kStageBytes);
@@ -48,10 +49,18 @@ __global__ void __launch_bounds__(32 * NW)
     const int b = blockIdx.x / p.CGB;
     const int64_t c0 = (int64_t)(blockIdx.x - b * p.CGB) * Cw;
     const int64_t T = p.T, C = p.C;
-    const int col = threadIdx.x * V;
+    const int col = threadIdx.x * 2;
     const int64_t c = c0 + col;
     const int64_t nchunks = (T + L - 1) / L;
 
+    // small per-channel loads first, so they do not queue behind the tiles
+    PairConsts cc;
+    pair_wu(p.w, p.u, c, C, cc);
+    St S[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+        S[j] = (p.state_in && c + j < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c + j)
+                                         : empty_state();
     if (threadIdx.x == 0) {
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
@@ -66,16 +75,9 @@ __global__ void __launch_bounds__(32 * NW)
             tma_load_3d(sv + st * L * Cw, &tmv, (int)c0, st * L, b, mbar + st);
         }
     }
-
-    ChanConsts cc[V];
-    channel_consts<V>(p.w, p.u, c, C, cc);
-    St S[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j)
-        S[j] = (p.state_in && c + j < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c + j)
-                                         : empty_state();
+    pair_derive(cc);
     IO* yg = static_cast<IO*>(p.y);
-    const bool vec_ok = c + V <= C;
+    const bool pair_ok = c + 2 <= C;
     bool failed = false;
 
     for (int64_t q = 0; q < nchunks; ++q) {
@@ -89,24 +91,24 @@ __global__ void __launch_bounds__(32 * NW)
         const int n = (int)min((int64_t)L, T - tq);
         const IO* kr = sk + st * L * Cw;
         const IO* vr = sv + st * L * Cw;
-        ChunkRegs<V, L> r;
-        St sum[V];
-        chunk_phase1<IO, V, L>(r, kr, vr, Cw, col, n, cc, sum);
+        PairRef r;
+        St sum[2];
         const int64_t ybase = ((int64_t)b * T + tq) * C + c;
-        auto out_one = [&](int i, int j, float yv) {
-            if (c + j < C) yg[ybase + (int64_t)i * C + j] = Io<IO>::from_f(yv);
+        auto out_one = [&](int i, int j, float y) {
+            if (c + j < C) yg[ybase + (int64_t)i * C + j] = Io<IO>::from_f(y);
         };
-        auto out_vec = [&](int i, const float (&yv)[V]) {
-            if (vec_ok) {
-                store_vec<IO, V>(yg + ybase + (int64_t)i * C, yv);
+        auto out_pair = [&](int i, f2 y) {
+            if (pair_ok) {
+                Pair<IO>::store(yg + ybase + (int64_t)i * C, y);
             } else {
-#pragma unroll
-                for (int j = 0; j < V; ++j) out_one(i, j, yv[j]);
+                out_one(i, 0, lo(y));
+                out_one(i, 1, hi(y));
             }
         };
-        chunk_phase3<IO, V, L>(r, kr, vr, Cw, col, n, S, cc, out_vec, out_one);
+        chunk_phase1<IO, L>(r, kr, vr, Cw, col, n, cc, sum);
+        chunk_phase3<IO, L>(r, kr, vr, Cw, col, n, S, cc, out_pair, out_one);
 #pragma unroll
-        for (int j = 0; j < V; ++j) S[j] = combine(S[j], sum[j], (double)n * cc[j].w2);
+        for (int j = 0; j < 2; ++j) S[j] = combine(S[j], sum[j], (double)n * cc.w2[j]);
         __syncthreads();  // stage st fully consumed
         if (threadIdx.x == 0 && q + NS < nchunks) {
             mbar_arrive_expect_tx(mbar + st, 2u * Sh::kStageBytes);
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(32 * NW)
     }
     if (p.state_out) {
 #pragma unroll
-        for (int j = 0; j < V; ++j)
+        for (int j = 0; j < 2; ++j)
             if (c + j < C) store_state_log2(p.state_out, p.BC, (int64_t)b * C + c + j, S[j]);
     }
 }
