@@ -153,16 +153,19 @@ def kernel_source_hash():
 
 
 def recorded_traffic(workload, variant):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel sources changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.txt),
+    or None when the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as f:
-            d = json.load(f)
-        e = d[f"{workload}/{variant}"]
-        if e["kernel_source_hash"] == kernel_source_hash():
-            return float(e["dram_bytes_per_launch"])
-    except Exception:
+            for line in f:
+                parts = line.split()
+                if not parts or parts[0].startswith("#") or parts[0] != f"{workload}/{variant}":
+                    continue
+                kv = dict(p.split("=", 1) for p in parts[1:] if "=" in p)
+                if kv.get("kernel_source_hash") == kernel_source_hash():
+                    return float(kv["dram_bytes_per_launch"])
+    except OSError:
         pass
     return None
 
@@ -182,6 +185,23 @@ def cpu_baseline(wl, x):
             "kind": "oracle",
             "sample": f"the whole workload ({wl.B}x{wl.T}x{wl.C}) x {reps} passes, fp64 C "
                       f"recurrence, {cores} threads over channels"}
+
+
+def max_over_ranks(ms: float, device=None) -> float:
+    """The slowest rank's time (every rank takes part; a no-op for one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(channel_steps_per_rank: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job G channel-steps/s: every rank processes its own batch (weak
+    scaling) and the job takes as long as its slowest rank."""
+    return world * channel_steps_per_rank * steps / (ms / 1e3) / 1e9
 
 
 def run_native(args):
@@ -264,11 +284,7 @@ def run_native(args):
     if world > 1:
         dist.barrier()
     clocks.stop()
-    ms = start.elapsed_time(end)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dev)
     if wkv4.device_error() != 0:
         raise RuntimeError("device-side wait ran out during the timed region")
 
@@ -306,12 +322,10 @@ def run_native(args):
                 e2e_step()
         e2.record(stream)
         torch.cuda.synchronize()
-        t2 = torch.tensor([s2.elapsed_time(e2)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        t2_ms = max_over_ranks(s2.elapsed_time(e2), dev)
         h2d = 2 * io_bytes(wl) + (12 * wl.B * wl.C if sih is not None else 0)
         d2h = io_bytes(wl) + 12 * wl.B * wl.C
-        e2e = {"value": world * wl.channel_steps * n_e2e / (float(t2.item()) / 1e3) / 1e9,
+        e2e = {"value": job_throughput(wl.channel_steps, n_e2e, world, t2_ms),
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": n_e2e}
 
@@ -321,7 +335,7 @@ def run_native(args):
         achieved = algorithmic_bytes(wl) / per_launch_s / 1e9
         line = {
             "metric": METRIC,
-            "value": world * wl.channel_steps * K / (ms / 1e3) / 1e9,
+            "value": job_throughput(wl.channel_steps, K, world, ms),
             "unit": UNIT,
             "n_gpus": world,
             "steps": K,

@@ -15,7 +15,8 @@ from typing import Optional, Tuple
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libwkv4.so")
+# WKV4_LIB selects another build of the library (e.g. one tuned differently)
+LIB_PATH = os.environ.get("WKV4_LIB") or os.path.join(_PKG, "libwkv4.so")
 
 F32, F16, BF16 = 0, 1, 2
 KERNEL_AUTO, KERNEL_SEQ, KERNEL_SCAN, KERNEL_SCAN_LDG, KERNEL_STEP = 0, 1, 2, 3, 4
