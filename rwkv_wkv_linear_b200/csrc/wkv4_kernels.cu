@@ -112,7 +112,7 @@ static cudaError_t scan_occupancy(int (&bps)[3]) {
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     for (int i = 0; i < 3; ++i) {
-        const ScanLayout<IO, L, NB> lay{kNwChoices[i]};
+        const ScanLayout<IO, L, NB> lay{kNwChoices[i], kMaxCluster};  // largest cluster: safe bound
         int v = (dev >= 0 && dev < 64) ? occ.bps[dev][i].load(std::memory_order_relaxed) : 0;
         if (v == 0) {
             v = -1;
@@ -180,7 +180,7 @@ static cudaError_t launch_scan_nb(const FwdArgs& a, const CUtensorMap& tk, const
                                   const CUtensorMap& ty, const ScanParams& p, const ScanShape& sh,
                                   int64_t tiles) {
     auto kern = wkv4_scan_kernel<IO, L, NB, kTMA>;
-    const ScanLayout<IO, L, NB> lay{sh.nw};
+    const ScanLayout<IO, L, NB> lay{sh.nw, sh.nc};
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(tiles * sh.nc), 1, 1);

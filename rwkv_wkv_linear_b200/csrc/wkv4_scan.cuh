@@ -10,12 +10,11 @@
 // starts as soon as its rows land.  Per round:
 //   1. every warp summarises its chunk from the empty state (chunk_phase1);
 //   2. warp 0 scans the NW chunk summaries (the state contribution before
-//      each chunk, the segment's aggregate) and publishes the aggregate in
-//      its CTA's shared memory;
-//   3. one cluster barrier; the warps copy the NC aggregates of the round from
-//      the cluster's shared memory (DSMEM loads, all in flight together) and
-//      warp 0 folds them, from the state carried into the round, into the
-//      state at the segment start and the state carried into the next round;
+//      each chunk, the segment's aggregate) and pushes the aggregate into the
+//      shared memory of every CTA of the cluster (DSMEM stores, posted);
+//   3. one cluster barrier; every warp folds the NC aggregates of the round,
+//      from the state carried into the round, into the state at the segment
+//      start and the state carried into the next round;
 //   4. every warp emits its chunk's outputs (chunk_phase3) into its k rows
 //      and sends them out with its own TMA store.
 // With several rounds the next round's rows are prefetched into a second
@@ -50,13 +49,14 @@ struct ScanLayout {
     __host__ __device__ size_t tile() const { return (size_t)nw * kChunkBytes; }
     __host__ __device__ size_t k(int buf) const { return (size_t)buf * 2 * tile(); }
     __host__ __device__ size_t v(int buf) const { return k(buf) + tile(); }
-    __host__ __device__ size_t sums() const { return (size_t)NB * 2 * tile(); }       // [nw][Cg] x 16 B
-    __host__ __device__ size_t agg() const { return sums() + (size_t)nw * kCg * 16; }  // [2][Cg] x 16 B
-    __host__ __device__ size_t start() const { return agg() + (size_t)2 * kCg * 16; }  // [Cg] x 16 B
-    __host__ __device__ size_t peers() const { return start() + (size_t)kCg * 16; }    // [8][Cg] x 16 B
-    __host__ __device__ size_t params() const { return peers() + (size_t)8 * kCg * 16; } // w, u, state [5][Cg] f32
-    __host__ __device__ size_t bars() const { return params() + (size_t)5 * kCg * 4; }  // [NB][nw] + 1 x 8 B
-    __host__ __device__ size_t bytes() const { return 1024 + bars() + (size_t)(NB * nw + 1) * 8; }
+    int nc;
+    __host__ __device__ size_t sums() const { return (size_t)NB * 2 * tile(); }        // [nw][Cg] x 16 B
+    __host__ __device__ size_t params() const { return sums() + (size_t)nw * kCg * 16; }  // w, u, state [5][Cg] f32
+    __host__ __device__ size_t bars() const { return params() + (size_t)5 * kCg * 4; }    // [NB][nw] + 1 x 8 B
+    __host__ __device__ size_t agg() const {                                              // [2][nc][Cg] x 16 B
+        return (bars() + (size_t)(NB * nw + 1) * 8 + 15) & ~(size_t)15;
+    }
+    __host__ __device__ size_t bytes() const { return 1024 + agg() + (size_t)2 * nc * kCg * 16; }
 };
 
 struct ScanParams {
@@ -100,7 +100,9 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     constexpr int Cg = ScanLayout<IO, L, NB>::kCg;
     constexpr int kChunkBytes = ScanLayout<IO, L, NB>::kChunkBytes;
     const int NW = blockDim.x >> 5;
-    const ScanLayout<IO, L, NB> lay{NW};
+    cg::cluster_group cluster = cg::this_cluster();
+    const int NC = (int)cluster.num_blocks();
+    const ScanLayout<IO, L, NB> lay{NW, NC};
     const int Ts = NW * L;
     extern __shared__ unsigned char smem_raw[];
     // align by offsetting the shared array itself (a round trip through an
@@ -109,8 +111,6 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     const TripleRef sums = triples(base + lay.sums(), NW * Cg);      // [NW][Cg]
     uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // [NB][NW]
 
-    cg::cluster_group cluster = cg::this_cluster();
-    const int NC = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     const int g = blockIdx.x / NC;
     const int b = g / p.CGB;
@@ -142,7 +142,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     // with aligned pointers comes by bulk copy on its own mbarrier, issued
     // before the tiles, so it does not queue behind other CTAs' tile traffic.
     PairConsts cc;
-    St carry[2];  // warp 0: the state carried into the current round
+    St carry[2];  // every warp: the state carried into the current round
     uint64_t* pbar = mbar + NB * NW;
     float* sw = reinterpret_cast<float*>(base + lay.params());  // [5][Cg]: w, u, a, b, p
     const bool bulk = kTMA && p.bulk_params && c0 + Cg <= C;
@@ -163,13 +163,11 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         }
     } else {
         pair_wu(p.w, p.u, c0 + col, C, cc);
-        if (warp == 0) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int64_t c = c0 + col + j;
-                carry[j] = (p.state_in && c < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c)
-                                                 : empty_state();
-            }
+        for (int j = 0; j < 2; ++j) {
+            const int64_t c = c0 + col + j;
+            carry[j] = (p.state_in && c < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c)
+                                             : empty_state();
         }
     }
     if constexpr (kTMA) {
@@ -194,10 +192,9 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         for (int j = 0; j < 2; ++j) {
             cc.w[j] = sw[col + j];
             cc.u[j] = sw[Cg + col + j];
-            if (warp == 0)
-                carry[j] = p.state_in ? St{sw[2 * Cg + col + j], sw[3 * Cg + col + j],
-                                           (double)sw[4 * Cg + col + j] * kLog2eD}
-                                      : empty_state();
+            carry[j] = p.state_in ? St{sw[2 * Cg + col + j], sw[3 * Cg + col + j],
+                                       (double)sw[4 * Cg + col + j] * kLog2eD}
+                                  : empty_state();
         }
     }
     pair_derive(cc);
@@ -242,11 +239,11 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         for (int j = 0; j < 2; ++j) sums.put(warp * Cg + col + j, sum[j]);
         __syncthreads();
 
-        // ---- 2. warp 0: exclusive prefix of the chunk summaries (in place)
-        //         and the segment aggregate
+        // ---- 2. warp 0: exclusive prefix of the chunk summaries (in place); the
+        //         segment aggregate is pushed into slot [round & 1][rank] of every
+        //         CTA of the cluster (posted remote stores)
         const int slot = round & 1;
-        const TripleRef agg = triples(base + lay.agg() + (size_t)slot * Cg * 16, Cg);
-        const TripleRef start = triples(base + lay.start(), Cg);
+        const TripleRef agg = triples(base + lay.agg() + (size_t)slot * NC * Cg * 16, NC * Cg);
         if (warp == 0) {
             St acc[2] = {empty_state(), empty_state()};
 #pragma unroll 1
@@ -260,47 +257,38 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                     acc[j] = combine(acc[j], Sq, nq * cc.w2[j]);
                 }
             }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) agg.put(col + j, acc[j]);
-        }
-
-        // ---- 3. copy the cluster's aggregates of this round into local shared
-        //         memory (warp q reads peers q, q + NW, ...: the remote loads of
-        //         all warps are in flight together); warp 0 folds them
-        cluster.sync();
-        for (int q = warp; q < NC; q += NW) {
-            const float* ra = cluster.map_shared_rank(agg.a, q);
-            const float* rb = cluster.map_shared_rank(agg.b, q);
-            const double* rp = cluster.map_shared_rank(agg.p, q);
-            const TripleRef dst = triples(base + lay.peers() + (size_t)q * Cg * 16, Cg);
-            const float2 a2 = *reinterpret_cast<const float2*>(ra + col);
-            const float2 b2 = *reinterpret_cast<const float2*>(rb + col);
-            const double p0 = rp[col], p1 = rp[col + 1];
-            dst.put(col, {a2.x, b2.x, p0});
-            dst.put(col + 1, {a2.y, b2.y, p1});
-        }
-        __syncthreads();
-        if (warp == 0) {
+            const int off = rank * Cg + col;
 #pragma unroll 1
             for (int q = 0; q < NC; ++q) {
-                const TripleRef src = triples(base + lay.peers() + (size_t)q * Cg * 16, Cg);
-                const int64_t sq = t0 + (int64_t)(q - rank) * Ts;
-                const double nq = (double)max((int64_t)0, min((int64_t)Ts, T - sq));
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    if (q == rank) start.put(col + j, carry[j]);
-                    carry[j] = combine(carry[j], src.get(col + j), nq * cc.w2[j]);
-                }
+                float* ra = cluster.map_shared_rank(agg.a, q);
+                float* rb = cluster.map_shared_rank(agg.b, q);
+                double* rp = cluster.map_shared_rank(agg.p, q);
+                *reinterpret_cast<float2*>(ra + off) = make_float2(acc[0].a, acc[1].a);
+                *reinterpret_cast<float2*>(rb + off) = make_float2(acc[0].b, acc[1].b);
+                rp[off] = acc[0].p;
+                rp[off + 1] = acc[1].p;
             }
         }
-        __syncthreads();
+
+        // ---- 3. every warp folds the round's aggregates from its own shared memory
+        cluster.sync();
+        St P[2];
+#pragma unroll 1
+        for (int q = 0; q < NC; ++q) {
+            const int64_t sq = t0 + (int64_t)(q - rank) * Ts;
+            const double nq = (double)max((int64_t)0, min((int64_t)Ts, T - sq));
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if (q == rank) P[j] = carry[j];
+                carry[j] = combine(carry[j], agg.get(q * Cg + col + j), nq * cc.w2[j]);
+            }
+        }
 
         // ---- 4. outputs of this warp's chunk
         St S[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-            S[j] = combine(start.get(col + j), sums.get(warp * Cg + col + j),
-                           (double)(warp * L) * cc.w2[j]);
+            S[j] = combine(P[j], sums.get(warp * Cg + col + j), (double)(warp * L) * cc.w2[j]);
         if constexpr (kTMA) {
             // y is staged in place of k (step i reads k_i before writing y_i)
             auto out_pair = [=](int i, f2 y) { Pair<IO>::store(kr + i * Cg + col, y); };
@@ -345,8 +333,8 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     if constexpr (kTMA) {
         if (lane == 0) bulk_wait_read_all();  // the staged rows stay valid until read
     }
-    // peers may still be reading this CTA's aggregates
-    cluster.sync();
+    // No barrier before leaving: peers only write into this CTA's shared
+    // memory before a round's cluster barrier, and read only their own.
 }
 
 }  // namespace wkv4
