@@ -105,17 +105,7 @@ int cuda_status(cudaError_t e) {
 }
 
 int run_scan(const FwdArgs& a, bool want_tma) {
-    const bool tma = want_tma && tma_eligible(a);
-    CUtensorMap tk, tv, ty;
-    if (tma) {
-        const wkv4::Geom g = wkv4::scan_geom(a.dtype);
-        if (!encode_btc(&tk, a.k, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t) ||
-            !encode_btc(&tv, a.v, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t) ||
-            !encode_btc(&ty, a.y, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t))
-            return WKV4_ERR_CUDA;
-    }
-    return cuda_status(wkv4::launch_scan(a, tma ? &tk : nullptr, tma ? &tv : nullptr,
-                                         tma ? &ty : nullptr));
+    return cuda_status(wkv4::launch_scan(a, want_tma && tma_eligible(a), encode_btc));
 }
 
 int run_seq(const FwdArgs& a) {

@@ -24,6 +24,7 @@ __device__ __forceinline__ f2 pk(float lo, float hi) {
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
     return r;
 }
+__device__ __forceinline__ f2 pku(uint32_t lo, uint32_t hi) { return ((f2)hi << 32) | lo; }
 __device__ __forceinline__ float lo(f2 r) { return __uint_as_float((unsigned)(r & 0xffffffffull)); }
 __device__ __forceinline__ float hi(f2 r) { return __uint_as_float((unsigned)(r >> 32)); }
 __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
@@ -229,9 +230,18 @@ struct PairRef {
 // Summary of the chunk from the empty state: max/min pass, then e_i and the
 // two Horner chains.  kFull (n == L) is a separate instantiation so that the
 // full chunk's loops carry no per-step guard and consecutive steps overlap.
-template <typename IO, int L, bool kFull>
+//
+// With kStash the pass also leaves, for the output pass,
+// each step's chunk-local numerator and denominator of y_i at the reference,
+//   N_i = A_i + e^u e_i v_i,   Dn_i = D_i + e^u e_i
+// (A_i, D_i: the chunk's state before step i, from the empty state), in
+// tensor memory at taddr: 4 columns a step (N lo, N hi, Dn lo, Dn hi), so
+// that the output pass needs neither k, v nor an exponential.
+template <typename IO, int L, bool kFull, bool kStash>
 __device__ __forceinline__ void chunk_phase1_t(PairRef& r, const IO* sk, const IO* sv, int stride,
-                                               int col, int n, const PairConsts& cc, St (&sum)[2]) {
+                                               int col, int n, const PairConsts& cc, St (&sum)[2],
+                                               uint32_t taddr) {
+    static_assert(!kStash || L % 4 == 0, "stash: whole column groups");
     typename Pair<IO>::Raw mx = Pair<IO>::raw(sk + col), mn = mx;
 #pragma unroll
     for (int i = 1; i < L; ++i)
@@ -246,14 +256,28 @@ __device__ __forceinline__ void chunk_phase1_t(PairRef& r, const IO* sk, const I
     const f2 l2e = pk(kLog2e, kLog2e);
     const f2 nref = pk(-r.kref[0], -r.kref[1]);
     f2 A = 0ull, D = 0ull;
+    uint32_t st[16];
+    if constexpr (kStash) __syncwarp();  // tensor-memory stores are warp-collective
 #pragma unroll
     for (int i = 0; i < L; ++i) {
         if (kFull || i < n) {
             const f2 e = ex2_2(fma2(Pair<IO>::load(sk + i * stride + col), l2e, nref));
-            A = fma2(cc.ew, A, mul2(e, Pair<IO>::load(sv + i * stride + col)));
+            const f2 ev = mul2(e, Pair<IO>::load(sv + i * stride + col));
+            if constexpr (kStash) {
+                const f2 N = fma2(cc.eu, ev, A), Dn = fma2(cc.eu, e, D);
+                const int s = (i & 3) * 4;
+                st[s] = (uint32_t)N;
+                st[s + 1] = (uint32_t)(N >> 32);
+                st[s + 2] = (uint32_t)Dn;
+                st[s + 3] = (uint32_t)(Dn >> 32);
+                // a group of 4 steps at a time (n is the same on every lane)
+                if ((i & 3) == 3 || (!kFull && i == n - 1)) tmem_st16(taddr + (uint32_t)(i >> 2) * 16u, st);
+            }
+            A = fma2(cc.ew, A, ev);
             D = fma2(cc.ew, D, e);
         }
     }
+    if constexpr (kStash) tmem_wait_st();
     const float Aj[2] = {lo(A), hi(A)}, Dj[2] = {lo(D), hi(D)};
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -265,13 +289,14 @@ __device__ __forceinline__ void chunk_phase1_t(PairRef& r, const IO* sk, const I
     }
 }
 
-template <typename IO, int L>
+template <typename IO, int L, bool kStash = false>
 __device__ __forceinline__ void chunk_phase1(PairRef& r, const IO* sk, const IO* sv, int stride,
-                                             int col, int n, const PairConsts& cc, St (&sum)[2]) {
+                                             int col, int n, const PairConsts& cc, St (&sum)[2],
+                                             uint32_t taddr = 0) {
     if (n >= L) {
-        chunk_phase1_t<IO, L, true>(r, sk, sv, stride, col, L, cc, sum);
+        chunk_phase1_t<IO, L, true, kStash>(r, sk, sv, stride, col, L, cc, sum, taddr);
     } else if (n > 0) {
-        chunk_phase1_t<IO, L, false>(r, sk, sv, stride, col, n, cc, sum);
+        chunk_phase1_t<IO, L, false, kStash>(r, sk, sv, stride, col, n, cc, sum, taddr);
     } else {
         sum[0] = sum[1] = empty_state();
         r.fast[0] = r.fast[1] = false;
@@ -348,6 +373,93 @@ __device__ __forceinline__ void chunk_phase3(const PairRef& r, const IO* sk, con
     } else {
         chunk_phase3_general<IO, L, OutOne>(r, sk, sv, stride, col, n, f3[0], f3[1], Ah, Dh, S[0],
                                             S[1], cc, out_one);
+    }
+}
+
+// Outputs of a chunk of n steps from the state S at its start by the exact
+// per-step max-trick, reading k and v of channel j at gk[i * stride + j],
+// gv[...] (global memory; only channels with ok[j]).  The fallback of the
+// stash path: it runs for a warp only where some lane's chunk leaves the
+// fixed-reference range.
+template <typename IO, typename OutOne>
+__device__ __noinline__ void chunk_exact_global(const IO* gk, const IO* gv, int64_t stride, int n,
+                                                bool ok0, bool ok1, St S0, St S1,
+                                                const PairConsts& cc, OutOne out_one) {
+    const bool ok[2] = {ok0, ok1};
+    const St S[2] = {S0, S1};
+    for (int j = 0; j < 2; ++j) {
+        if (!ok[j]) continue;
+        St s = S[j];
+        const double u2 = (double)cc.u[j] * kLog2eD;
+        for (int i = 0; i < n; ++i) {
+            const float k = Io<IO>::to_f(gk[(int64_t)i * stride + j]);
+            const float v = Io<IO>::to_f(gv[(int64_t)i * stride + j]);
+            out_one(i, j, exact_step(s, k, v, cc.w2[j], u2));
+        }
+    }
+}
+
+// Outputs of a chunk of n steps whose summary pass left its stash in tensor
+// memory at taddr (chunk_phase1 with kStash).  When every lane of the warp
+// has both channels on the fixed-reference path (the decision is warp-wide:
+// tensor-memory loads are warp-collective), from the state (alpha, beta) at
+// the chunk start rescaled to the reference,
+//   y_i = (e^{i w} alpha + N_i) / (e^{i w} beta + Dn_i),
+// one reciprocal a step, through out_pair(i, y); otherwise the exact per-step
+// path from k, v in global memory (gk, gv: the pair's first channel at the
+// chunk's first step, row stride `stride`; ok[j]: channel j exists) through
+// out_one(i, j, y).
+template <typename IO, int L, typename OutPair, typename OutOne>
+__device__ __forceinline__ void chunk_phase3_stash(const PairRef& r, int n, const St (&S)[2],
+                                                   const PairConsts& cc, uint32_t taddr,
+                                                   const IO* gk, const IO* gv, int64_t stride,
+                                                   bool ok0, bool ok1, OutPair out_pair,
+                                                   OutOne out_one) {
+    static_assert(L % 4 == 0, "stash: whole column groups");
+    if (n <= 0) return;
+    bool f3[2];
+    float a0[2], b0[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const double lift = S[j].p - (double)r.kref[j];
+        f3[j] = r.fast[j] && (lift <= (double)(kFastStateLift * kLog2e));
+        const float sc = ex2((float)lift);
+        a0[j] = S[j].a * sc;
+        b0[j] = S[j].b * sc;
+    }
+    if (__all_sync(0xffffffffu, f3[0] && f3[1])) {
+        const f2 al = pk(a0[0], a0[1]), be = pk(b0[0], b0[1]);
+        f2 f = pk(1.f, 1.f);  // e^{i w}
+        if (n == L) {
+#pragma unroll
+            for (int q = 0; q < L / 4; ++q) {
+                uint32_t st[16];
+                tmem_ld16(taddr + (uint32_t)q * 16u, st);
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const f2 N = pku(st[4 * s], st[4 * s + 1]), Dn = pku(st[4 * s + 2], st[4 * s + 3]);
+                    out_pair(4 * q + s, mul2(fma2(f, al, N), rcp2(fma2(f, be, Dn))));
+                    f = mul2(f, cc.ew);
+                }
+            }
+        } else {
+#pragma unroll 1
+            for (int q = 0; 4 * q < n; ++q) {
+                uint32_t st[16];
+                tmem_ld16(taddr + (uint32_t)q * 16u, st);
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    if (4 * q + s < n) {
+                        const f2 N = pku(st[4 * s], st[4 * s + 1]);
+                        const f2 Dn = pku(st[4 * s + 2], st[4 * s + 3]);
+                        out_pair(4 * q + s, mul2(fma2(f, al, N), rcp2(fma2(f, be, Dn))));
+                        f = mul2(f, cc.ew);
+                    }
+                }
+            }
+        }
+    } else {
+        chunk_exact_global<IO>(gk, gv, stride, n, ok0, ok1, S[0], S[1], cc, out_one);
     }
 }
 

@@ -30,13 +30,17 @@ struct Geom {
     size_t smem;    // dynamic shared memory per CTA (bytes)
 };
 
-Geom scan_geom(int dtype);
 Geom seq_geom(int dtype);
 size_t dtype_size(int dtype);
 
-// Launchers.  Tensor maps are NULL for the element-wise (LDG) variant.
-cudaError_t launch_scan(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
-                        const CUtensorMap* ty);
+// Encoder of a 3-D [B][T][C] tensor map with a box of box_c channels x
+// box_t steps (false on failure).
+typedef bool (*EncodeFn)(CUtensorMap* map, const void* ptr, int dtype, int64_t B, int64_t T,
+                         int64_t C, int box_c, int box_t);
+
+// Launchers.  The scan picks its shape, then encodes its tensor maps with
+// `encode` (tma) or loads element-wise (!tma).
+cudaError_t launch_scan(const FwdArgs& a, bool tma, EncodeFn encode);
 cudaError_t launch_seq(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv);
 cudaError_t launch_step(const FwdArgs& a);     // exact per-step kernel, any T >= 1
 cudaError_t launch_decode(const FwdArgs& a);   // T == 1, vectorised when aligned

@@ -18,6 +18,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <climits>
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
@@ -36,11 +38,8 @@ __device__ unsigned int g_device_error = 0;
 
 namespace wkv4 {
 
-// Kernel configurations: chunk length L per dtype for the scan (a warp's
-// rows are L steps x 64 channels); <IO, L, NW, NS> for the sequential kernel
-// (64*NW channels, NS stages of L steps).
-constexpr int kScanL16 = 32;  // 16-bit I/O
-constexpr int kScanL32 = 16;  // fp32 I/O
+// Sequential kernel configurations <IO, L, NW, NS>: 64 NW channels, NS
+// stages of L steps.
 #define WKV4_SEQ_F32 float, 16, 2, 4
 #define WKV4_SEQ_F16 __half, 16, 4, 4
 #define WKV4_SEQ_BF16 __nv_bfloat16, 16, 4, 4
@@ -70,12 +69,6 @@ static Geom seq_geom_t() {
     return {Sh::kCw, L, Sh::kThreads, Sh::kSmem};
 }
 
-// TMA boxes: a scan box is one warp's rows (64 channels x L steps).
-Geom scan_geom(int dtype) {
-    const int L = dtype == WKV4_F32 ? kScanL32 : kScanL16;
-    return {64, L, 0, 0};
-}
-
 Geom seq_geom(int dtype) {
     if (dtype == WKV4_F32) return seq_geom_t<WKV4_SEQ_F32>();
     if (dtype == WKV4_F16) return seq_geom_t<WKV4_SEQ_F16>();
@@ -94,16 +87,42 @@ static int env_int(const char* name, int dflt) {
 }
 
 constexpr size_t kMaxSmem = 227 * 1024;
-constexpr int kNwChoices[3] = {4, 8, 16};
+constexpr int kTmemColumns = 512;  // tensor-memory columns per SM
+
+// Dynamic shared memory to request for a scan CTA: its layout's bytes, raised
+// where needed so that no more CTAs fit on an SM than the SM's tensor memory
+// serves (a CTA allocates `cols` columns at its start and holds them to its
+// end; an allocation that cannot be met would wait for another CTA's release).
+static size_t scan_smem_request(size_t bytes, int cols) {
+    int dev = 0, per_sm = 233472, reserved = 1024;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    }
+    const int cap = kTmemColumns / cols;  // CTAs per SM the tensor memory serves
+    // (cap + 1) CTAs of (request + reserved) bytes each do not fit on an SM
+    const size_t floor_bytes = (size_t)per_sm / (size_t)(cap + 1) + 1;
+    size_t need = floor_bytes > (size_t)reserved ? floor_bytes - (size_t)reserved : 0;
+    need = (need + 127) & ~(size_t)127;
+    return bytes > need ? bytes : need;
+}
+
+// Scan configuration per I/O type: steps per warp chunk (a warp's rows are
+// L steps x 64 channels).
+template <typename IO> struct ScanL { static constexpr int L = 32; };
+template <> struct ScanL<float> { static constexpr int L = 16; };
+
+constexpr int kNwChoices[2] = {8, 4};  // warps per CTA, in order of preference
 
 // Resident CTAs per SM of one scan instantiation for each warp count, cached
-// per device (0 = that warp count does not fit).
+// per device (0: that warp count does not fit, or more CTAs would share an
+// SM than its tensor memory serves).
 struct ScanOcc {
-    std::atomic<int> bps[64][3];
+    std::atomic<int> bps[64][2];
 };
 
 template <typename IO, int L, int NB, bool kTMA>
-static cudaError_t scan_occupancy(int (&bps)[3]) {
+static cudaError_t scan_occupancy(int (&bps)[2]) {
     static DeviceFlags attr;
     static ScanOcc occ;
     auto kern = wkv4_scan_kernel<IO, L, NB, kTMA>;
@@ -111,48 +130,47 @@ static cudaError_t scan_occupancy(int (&bps)[3]) {
     if (e != cudaSuccess) return e;
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    for (int i = 0; i < 3; ++i) {
-        const ScanLayout<IO, L, NB> lay{kNwChoices[i], kMaxCluster};  // largest cluster: safe bound
-        int v = (dev >= 0 && dev < 64) ? occ.bps[dev][i].load(std::memory_order_relaxed) : 0;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    for (int i = 0; i < 2; ++i) {
+        int v = occ.bps[dev][i].load(std::memory_order_acquire);
         if (v == 0) {
             v = -1;
-            if (lay.bytes() <= kMaxSmem) {
+            // the largest cluster's layout: a bound for every cluster size
+            const ScanLayout<IO, L, NB> lay{kNwChoices[i], kMaxCluster};
+            const size_t req = scan_smem_request(lay.bytes(), lay.tmem_cols());
+            if (req <= kMaxSmem) {
                 int n = 0;
                 if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * kNwChoices[i],
-                                                                       lay.bytes())) != cudaSuccess)
+                                                                       req)) != cudaSuccess)
                     return e;
-                v = n > 0 ? n : -1;
+                if (n > 0 && n * lay.tmem_cols() <= kTmemColumns) v = n;
             }
-            if (dev >= 0 && dev < 64) occ.bps[dev][i].store(v, std::memory_order_relaxed);
+            occ.bps[dev][i].store(v, std::memory_order_release);
         }
         bps[i] = v > 0 ? v : 0;
     }
     return cudaSuccess;
 }
 
-// Launch shape of the scan: warps per CTA (NW) and cluster size (NC).
-// Measured on B200 (169m- and 14B-width prefill, 65536-step fp32): 8 warps
-// per CTA is best wherever it fits.  When T fits in at most 8 segments, one
-// round with NC = segments (rounded up to a power of two) wins even if the
-// grid takes several waves; when T needs several rounds, a second wave of
-// CTAs that each walk all of T is costly, so NC is the largest power of two
-// whose grid still fits in one wave.  WKV4_SCAN_NW / WKV4_SCAN_CLUSTER
-// override (tuning).
+// Launch shape of the scan: warps per CTA (NW) and cluster size (NC).  8 warps
+// per CTA wherever it fits.  When T fits in at most 8 segments, one round
+// with NC = segments (rounded up to a power of two), even if the grid takes
+// several waves; when T needs several rounds, NC is the largest power of two
+// whose grid still fits in one wave (a second wave of CTAs that each walk all
+// of T would be costly).  WKV4_SCAN_NW / WKV4_SCAN_CLUSTER override (tuning).
 struct ScanShape {
     int nw, nc, rounds, nb;
 };
 
 template <typename IO, int L, bool kTMA>
 static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
-    int b1[3], b2[3];
+    int b1[2], b2[2];
     cudaError_t e = scan_occupancy<IO, L, 1, kTMA>(b1);
     if (e != cudaSuccess) return e;
     if ((e = scan_occupancy<IO, L, 2, kTMA>(b2)) != cudaSuccess) return e;
     const int sms = sm_count();
     const int force_nw = env_int("WKV4_SCAN_NW", 0), force_nc = env_int("WKV4_SCAN_CLUSTER", 0);
-    static const int kNwOrder[3] = {1, 2, 0};  // indices into kNwChoices: 8, 16, 4
-    for (int oi = 0; oi < 3; ++oi) {
-        const int i = kNwOrder[oi];
+    for (int i = 0; i < 2; ++i) {
         const int nw = kNwChoices[i];
         if (force_nw && nw != force_nw) continue;
         const int64_t nseg = (T + (int64_t)nw * L - 1) / ((int64_t)nw * L);
@@ -162,12 +180,12 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
         } else if (nseg <= kMaxCluster) {
             while (nc < nseg) nc *= 2;
         } else {
-            const int bps = b2[i];
-            const int64_t cap = (int64_t)bps * sms;
+            const int64_t cap = (int64_t)b2[i] * sms;
             while (nc < kMaxCluster && tiles * nc * 2 <= cap) nc *= 2;
         }
         const int64_t rounds = (nseg + nc - 1) / nc;
-        const int nb = rounds > 1 ? 2 : 1;
+        if (rounds > (1ll << 30)) continue;
+        const int nb = (kTMA && rounds > 1) ? 2 : 1;
         if ((nb == 1 ? b1[i] : b2[i]) <= 0) continue;  // does not fit on an SM
         out = {nw, nc, (int)rounds, nb};
         return cudaSuccess;
@@ -176,16 +194,25 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
 }
 
 template <typename IO, int L, int NB, bool kTMA>
-static cudaError_t launch_scan_nb(const FwdArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                                  const CUtensorMap& ty, const ScanParams& p, const ScanShape& sh,
-                                  int64_t tiles) {
+static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const ScanShape& sh,
+                                  int64_t tiles, EncodeFn encode) {
+    CUtensorMap tk, tv, ty;
+    std::memset(&tk, 0, sizeof(tk));
+    std::memset(&tv, 0, sizeof(tv));
+    std::memset(&ty, 0, sizeof(ty));
+    if (kTMA) {
+        if (!encode(&tk, a.k, a.dtype, a.B, a.T, a.C, 64, L) ||
+            !encode(&tv, a.v, a.dtype, a.B, a.T, a.C, 64, L) ||
+            !encode(&ty, a.y, a.dtype, a.B, a.T, a.C, 64, L))
+            return cudaErrorInvalidValue;
+    }
     auto kern = wkv4_scan_kernel<IO, L, NB, kTMA>;
     const ScanLayout<IO, L, NB> lay{sh.nw, sh.nc};
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(tiles * sh.nc), 1, 1);
     cfg.blockDim = dim3(32 * sh.nw, 1, 1);
-    cfg.dynamicSmemBytes = lay.bytes();
+    cfg.dynamicSmemBytes = scan_smem_request(lay.bytes(), lay.tmem_cols());
     cfg.stream = a.stream;
     cudaLaunchAttribute attrs[1];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
@@ -197,9 +224,9 @@ static cudaError_t launch_scan_nb(const FwdArgs& a, const CUtensorMap& tk, const
     return cudaLaunchKernelEx(&cfg, kern, tk, tv, ty, p);
 }
 
-template <typename IO, int L, bool kTMA>
-static cudaError_t launch_scan_t(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
-                                 const CUtensorMap* ty) {
+template <typename IO, bool kTMA>
+static cudaError_t launch_scan_t(const FwdArgs& a, EncodeFn encode) {
+    constexpr int L = ScanL<IO>::L;
     ScanParams p{};
     p.T = a.T;
     p.C = a.C;
@@ -218,29 +245,21 @@ static cudaError_t launch_scan_t(const FwdArgs& a, const CUtensorMap* tk, const 
     ScanShape sh;
     cudaError_t e = pick_scan_shape<IO, L, kTMA>(tiles, a.T, sh);
     if (e != cudaSuccess) return e;
+    if (tiles * sh.nc > (int64_t)INT32_MAX) return cudaErrorInvalidConfiguration;
     p.rounds = sh.rounds;
-    CUtensorMap dummy;
-    std::memset(&dummy, 0, sizeof(dummy));
-    const CUtensorMap& mk = tk ? *tk : dummy;
-    const CUtensorMap& mv = tv ? *tv : dummy;
-    const CUtensorMap& my = ty ? *ty : dummy;
-    if (sh.nb == 1) return launch_scan_nb<IO, L, 1, kTMA>(a, mk, mv, my, p, sh, tiles);
-    return launch_scan_nb<IO, L, 2, kTMA>(a, mk, mv, my, p, sh, tiles);
+    if (sh.nb == 1) return launch_scan_nb<IO, L, 1, kTMA>(a, p, sh, tiles, encode);
+    return launch_scan_nb<IO, L, 2, kTMA>(a, p, sh, tiles, encode);
 }
 
-cudaError_t launch_scan(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
-                        const CUtensorMap* ty) {
-    const bool tma = tk != nullptr;
+cudaError_t launch_scan(const FwdArgs& a, bool tma, EncodeFn encode) {
     switch (a.dtype) {
         case WKV4_F32:
-            return tma ? launch_scan_t<float, kScanL32, true>(a, tk, tv, ty)
-                       : launch_scan_t<float, kScanL32, false>(a, tk, tv, ty);
+            return tma ? launch_scan_t<float, true>(a, encode) : launch_scan_t<float, false>(a, encode);
         case WKV4_F16:
-            return tma ? launch_scan_t<__half, kScanL16, true>(a, tk, tv, ty)
-                       : launch_scan_t<__half, kScanL16, false>(a, tk, tv, ty);
+            return tma ? launch_scan_t<__half, true>(a, encode) : launch_scan_t<__half, false>(a, encode);
         default:
-            return tma ? launch_scan_t<__nv_bfloat16, kScanL16, true>(a, tk, tv, ty)
-                       : launch_scan_t<__nv_bfloat16, kScanL16, false>(a, tk, tv, ty);
+            return tma ? launch_scan_t<__nv_bfloat16, true>(a, encode)
+                       : launch_scan_t<__nv_bfloat16, false>(a, encode);
     }
 }
 

@@ -8,18 +8,21 @@
 // whole T is one round of one wave.  Inside a CTA each warp owns one chunk of
 // L steps; its rows arrive by their own TMA box and mbarrier, so a warp
 // starts as soon as its rows land.  Per round:
-//   1. every warp summarises its chunk from the empty state (chunk_phase1);
+//   1. every warp summarises its chunk from the empty state (chunk_phase1
+//      with stash: the per-step numerators and denominators of its outputs
+//      go to tensor memory);
 //   2. warp 0 scans the NW chunk summaries (the state contribution before
 //      each chunk, the segment's aggregate) and pushes the aggregate into the
-//      shared memory of every CTA of the cluster (DSMEM stores, posted);
+//      shared memory of every CTA of the cluster (DSMEM stores);
 //   3. one cluster barrier; every warp folds the NC aggregates of the round,
 //      from the state carried into the round, into the state at the segment
 //      start and the state carried into the next round;
-//   4. every warp emits its chunk's outputs (chunk_phase3) into its k rows
+//   4. every warp computes its chunk's outputs from the stash into its k rows
 //      and sends them out with its own TMA store.
-// With several rounds the next round's rows are prefetched into a second
-// buffer (NB = 2).  There is no global scratch and no spin-wait on another
-// CTA: all exchange is through cluster shared memory and hardware barriers.
+// With several rounds the next round's rows are loaded into a second buffer
+// (NB = 2).
+// There is no global scratch and no spin-wait on another CTA: all exchange is
+// through cluster shared memory and hardware barriers.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -32,31 +35,36 @@ namespace cg = cooperative_groups;
 
 constexpr int kMaxCluster = 8;
 
-// Register cap of the scan kernel: enough CTAs per SM for the whole grid of
-// the common shapes to be resident at once.
+// Register cap of the scan kernel: two CTAs of 8 warps per SM.
 #ifndef WKV4_SCAN_MAXNREG
-#define WKV4_SCAN_MAXNREG 96
+#define WKV4_SCAN_MAXNREG 128
 #endif
 
-// Shared-memory layout for nw warps (offsets from a 1024-byte aligned base).
+// Shared-memory layout for nw warps and clusters of nc (offsets from a
+// 128-byte aligned base): NB row buffers of k and v, the chunk summaries,
+// the tile's w, u and state, barriers, two slots of aggregates.
 template <typename IO, int L, int NB>
 struct ScanLayout {
     static constexpr int kCg = 64;  // channels per tile: 32 lanes x 2
     static constexpr int kChunkBytes = L * kCg * (int)sizeof(IO);  // one warp's rows, one tensor
-    static_assert(L <= 256, "TMA box dims");
-    static_assert(kChunkBytes % 128 == 0, "TMA destination alignment");
-    int nw;
+    static constexpr int kAlign = 128;                               // TMA destinations
+    static_assert(L <= 256 && L % 4 == 0, "TMA box dims, stash column groups");
+    static_assert(kChunkBytes % kAlign == 0, "TMA destination alignment");
+    int nw, nc;
     __host__ __device__ size_t tile() const { return (size_t)nw * kChunkBytes; }
     __host__ __device__ size_t k(int buf) const { return (size_t)buf * 2 * tile(); }
     __host__ __device__ size_t v(int buf) const { return k(buf) + tile(); }
-    int nc;
-    __host__ __device__ size_t sums() const { return (size_t)NB * 2 * tile(); }        // [nw][Cg] x 16 B
-    __host__ __device__ size_t params() const { return sums() + (size_t)nw * kCg * 16; }  // w, u, state [5][Cg] f32
-    __host__ __device__ size_t bars() const { return params() + (size_t)5 * kCg * 4; }    // [NB][nw] + 1 x 8 B
-    __host__ __device__ size_t agg() const {                                              // [2][nc][Cg] x 16 B
-        return (bars() + (size_t)(NB * nw + 1) * 8 + 15) & ~(size_t)15;
+    __host__ __device__ size_t sums() const { return (size_t)NB * 2 * tile(); }          // [nw][Cg] x 16 B
+    __host__ __device__ size_t params() const { return sums() + (size_t)nw * kCg * 16; }  // [5][Cg] f32
+    __host__ __device__ size_t agg(int slot) const {                                    // [2][nc][Cg] x 16 B
+        return params() + (size_t)5 * kCg * 4 + (size_t)slot * nc * kCg * 16;
     }
-    __host__ __device__ size_t bytes() const { return 1024 + agg() + (size_t)2 * nc * kCg * 16; }
+    __host__ __device__ size_t bars() const { return agg(2); }  // rows [NB][nw], params x 8 B
+    __host__ __device__ size_t tslot() const { return bars() + (size_t)(NB * nw + 1) * 8; }
+    __host__ __device__ size_t bytes() const { return kAlign + tslot() + 8; }
+    // tensor-memory columns: 4 a step for each warp, warps w and w + 4
+    // sharing a lane quarter
+    __host__ __device__ int tmem_cols() const { return nw * L; }
 };
 
 struct ScanParams {
@@ -65,13 +73,13 @@ struct ScanParams {
     int rounds;  // ceil(segments / NC)
     const float* w;
     const float* u;
-    const void* k;  // element-wise variant only
+    const void* k;
     const void* v;
     const float* state_in;
     void* y;
     float* state_out;
     int64_t BC;
-    int bulk_params;  // w, u, state_in are 16-byte aligned: fetch them by bulk copy
+    int bulk_params;  // w, u, state_in 16-byte aligned and C % 4 == 0: bulk copies
 };
 
 // (a, b, p) triples in shared memory, stored as three planes of n entries.
@@ -93,23 +101,46 @@ __device__ __forceinline__ TripleRef triples(unsigned char* at, int n) {
     return {a, b, reinterpret_cast<double*>(b + n)};
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Split cluster barrier: every thread of every CTA of the cluster arrives,
+// then waits.  A releasing arrive publishes this thread's prior stores (the
+// DSMEM pushes) to the threads whose wait acquires; threads with nothing to
+// publish arrive relaxed.
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 template <typename IO, int L, int NB, bool kTMA>
 __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     wkv4_scan_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __grid_constant__ CUtensorMap tmy, const ScanParams p) {
-    constexpr int Cg = ScanLayout<IO, L, NB>::kCg;
-    constexpr int kChunkBytes = ScanLayout<IO, L, NB>::kChunkBytes;
+    using Lay = ScanLayout<IO, L, NB>;
+    constexpr int Cg = Lay::kCg;
+    constexpr int kChunkBytes = Lay::kChunkBytes;
+    constexpr unsigned kAlign = Lay::kAlign;
     const int NW = blockDim.x >> 5;
     cg::cluster_group cluster = cg::this_cluster();
     const int NC = (int)cluster.num_blocks();
-    const ScanLayout<IO, L, NB> lay{NW, NC};
+    const Lay lay{NW, NC};
     const int Ts = NW * L;
     extern __shared__ unsigned char smem_raw[];
     // align by offsetting the shared array itself (a round trip through an
     // integer would lose the address space and turn every access generic)
-    unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const TripleRef sums = triples(base + lay.sums(), NW * Cg);      // [NW][Cg]
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // [NB][NW]
+    unsigned char* base = smem_raw + ((kAlign - (smem_u32(smem_raw) & (kAlign - 1))) & (kAlign - 1));
+    const TripleRef sums = triples(base + lay.sums(), NW * Cg);       // [NW][Cg]
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // rows [NB][NW], params
+    uint64_t* pbar = mbar + NB * NW;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(base + lay.tslot());
+    float* sw = reinterpret_cast<float*>(base + lay.params());  // [5][Cg]: w, u, a, b, p
 
     const int rank = (int)cluster.block_rank();
     const int g = blockIdx.x / NC;
@@ -119,6 +150,9 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int col = lane * 2;
     const int64_t seg_stride = (int64_t)NC * Ts;  // steps per round
+    const IO* kg = static_cast<const IO*>(p.k);
+    const IO* vg = static_cast<const IO*>(p.v);
+    IO* yg = static_cast<IO*>(p.y);
 
     auto chunk_len = [&](int j, int q) -> int {  // steps of chunk q of this CTA in round j
         const int64_t tc = (int64_t)j * seg_stride + (int64_t)rank * Ts + (int64_t)q * L;
@@ -126,42 +160,59 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     };
     auto rows_k = [&](int buf) { return reinterpret_cast<IO*>(base + lay.k(buf)) + warp * L * Cg; };
     auto rows_v = [&](int buf) { return reinterpret_cast<IO*>(base + lay.v(buf)) + warp * L * Cg; };
-    auto issue_loads = [&](int j) {  // lane 0 of each warp: this warp's rows of round j
+    // Lane 0 of each warp: this warp's rows of round j into buffer j % NB.
+    // Every round completes one phase of the warp's barrier of that buffer (a
+    // plain arrive where nothing is copied), so its phases stay in step.
+    auto issue_rows = [&](int j) {
         if constexpr (kTMA) {
-            if (chunk_len(j, warp) <= 0) return;
+            if (j >= p.rounds) return;
             const int buf = j % NB;
-            const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
             uint64_t* bar = mbar + buf * NW + warp;
-            mbar_arrive_expect_tx(bar, 2u * kChunkBytes);
-            tma_load_3d(rows_k(buf), &tmk, (int)c0, t, b, bar);
-            tma_load_3d(rows_v(buf), &tmv, (int)c0, t, b, bar);
+            if (chunk_len(j, warp) > 0) {
+                const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
+                mbar_arrive_expect_tx(bar, 2u * kChunkBytes);
+                tma_load_3d(rows_k(buf), &tmk, (int)c0, t, b, bar);
+                tma_load_3d(rows_v(buf), &tmv, (int)c0, t, b, bar);
+            } else {
+                mbar_arrive(bar);
+            }
         }
     };
 
     // Per-channel w, u and the state for this tile: a full 64-channel slice
     // with aligned pointers comes by bulk copy on its own mbarrier, issued
-    // before the tiles, so it does not queue behind other CTAs' tile traffic.
+    // before the rows, so it does not queue behind other CTAs' row traffic.
+    const bool bulk = kTMA && p.bulk_params && c0 + Cg <= C;
+    if (warp == 0) tmem_alloc(tslot, (uint32_t)lay.tmem_cols());
+    if constexpr (kTMA) {
+        if (lane == 0) {
+            if (warp == 0) {
+                mbar_init(pbar, 1);
+                prefetch_tmap(&tmk);
+                prefetch_tmap(&tmv);
+                prefetch_tmap(&tmy);
+            }
+            for (int buf = 0; buf < NB; ++buf) mbar_init(mbar + buf * NW + warp, 1);
+            fence_mbar_init();
+            if (warp == 0 && bulk) {
+                const uint32_t nb = Cg * 4;
+                const int64_t ch = (int64_t)b * C + c0;
+                mbar_arrive_expect_tx(pbar, (p.state_in ? 5u : 2u) * nb);
+                bulk_load(sw, p.w + c0, nb, pbar);
+                bulk_load(sw + Cg, p.u + c0, nb, pbar);
+                if (p.state_in) {
+                    bulk_load(sw + 2 * Cg, p.state_in + ch, nb, pbar);
+                    bulk_load(sw + 3 * Cg, p.state_in + p.BC + ch, nb, pbar);
+                    bulk_load(sw + 4 * Cg, p.state_in + 2 * p.BC + ch, nb, pbar);
+                }
+            }
+            for (int j = 0; j < NB; ++j) issue_rows(j);
+        }
+        __syncwarp();
+    }
     PairConsts cc;
     St carry[2];  // every warp: the state carried into the current round
-    uint64_t* pbar = mbar + NB * NW;
-    float* sw = reinterpret_cast<float*>(base + lay.params());  // [5][Cg]: w, u, a, b, p
-    const bool bulk = kTMA && p.bulk_params && c0 + Cg <= C;
-    if (bulk) {
-        if (threadIdx.x == 0) {
-            mbar_init(pbar, 1);
-            fence_mbar_init();
-            const uint32_t nb = Cg * 4;
-            const int64_t ch = (int64_t)b * C + c0;
-            mbar_arrive_expect_tx(pbar, (p.state_in ? 5u : 2u) * nb);
-            bulk_load(sw, p.w + c0, nb, pbar);
-            bulk_load(sw + Cg, p.u + c0, nb, pbar);
-            if (p.state_in) {
-                bulk_load(sw + 2 * Cg, p.state_in + ch, nb, pbar);
-                bulk_load(sw + 3 * Cg, p.state_in + p.BC + ch, nb, pbar);
-                bulk_load(sw + 4 * Cg, p.state_in + 2 * p.BC + ch, nb, pbar);
-            }
-        }
-    } else {
+    if (!bulk) {
         pair_wu(p.w, p.u, c0 + col, C, cc);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -170,22 +221,20 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                                              : empty_state();
         }
     }
-    if constexpr (kTMA) {
-        if (lane == 0) {
-            if (warp == 0) {
-                prefetch_tmap(&tmk);
-                prefetch_tmap(&tmv);
-                prefetch_tmap(&tmy);
-            }
-            for (int buf = 0; buf < NB; ++buf) mbar_init(mbar + buf * NW + warp, 1);
-            fence_mbar_init();
-            for (int j = 0; j < NB && j < p.rounds; ++j) issue_loads(j);
-        }
-        __syncwarp();
-    }
+    // the tensor-memory base is in shared memory, every barrier initialised
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    // the CTAs of the cluster have all started before the first DSMEM store
+    // (this barrier's wait comes just before it)
+    cluster_arrive_relaxed();
+    const uint32_t tbase = *tslot;
+    // this warp's stash: its lane quarter, 4 L columns for each warp of the quarter
+    const uint32_t taddr = tbase + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((warp >> 2) * 4 * L);
+    bool failed = false;
     if (bulk) {
-        __syncthreads();  // the params barrier is initialised
         if (!mbar_wait_bounded(pbar, 0)) {
+            failed = true;
             if (lane == 0) atomicOr(&g_device_error, kErrTmaWait);
         }
 #pragma unroll
@@ -198,7 +247,6 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         }
     }
     pair_derive(cc);
-    bool failed = false;
 
     for (int round = 0; round < p.rounds; ++round) {
         const int buf = round % NB;
@@ -214,8 +262,6 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
             }
         } else {
             // element-wise loads of this warp's rows (any alignment, zero fill)
-            const IO* kg = static_cast<const IO*>(p.k);
-            const IO* vg = static_cast<const IO*>(p.v);
             for (int idx = lane; idx < L * Cg; idx += 32) {
                 const int rr = idx / Cg, ci = idx - rr * Cg;
                 const int64_t t = t0 + warp * L + rr, c = c0 + ci;
@@ -231,19 +277,20 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
             __syncwarp();
         }
 
-        // ---- 1. chunk summaries
+        // ---- 1. chunk summary and stash; then the rows are free
         PairRef ref;
         St sum[2];
-        chunk_phase1<IO, L>(ref, kr, vr, Cg, col, n, cc, sum);
+        chunk_phase1<IO, L, true>(ref, kr, vr, Cg, col, n, cc, sum, taddr);
 #pragma unroll
         for (int j = 0; j < 2; ++j) sums.put(warp * Cg + col + j, sum[j]);
         __syncthreads();
 
         // ---- 2. warp 0: exclusive prefix of the chunk summaries (in place); the
         //         segment aggregate is pushed into slot [round & 1][rank] of every
-        //         CTA of the cluster (posted remote stores)
+        //         CTA of the cluster
         const int slot = round & 1;
-        const TripleRef agg = triples(base + lay.agg() + (size_t)slot * NC * Cg * 16, NC * Cg);
+        const TripleRef agg = triples(base + lay.agg(slot), NC * Cg);
+        if (round == 0) cluster_wait();  // every CTA of the cluster has started
         if (warp == 0) {
             St acc[2] = {empty_state(), empty_state()};
 #pragma unroll 1
@@ -268,10 +315,13 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                 rp[off] = acc[0].p;
                 rp[off + 1] = acc[1].p;
             }
+            cluster_arrive_release();
+        } else {
+            cluster_arrive_relaxed();
         }
 
         // ---- 3. every warp folds the round's aggregates from its own shared memory
-        cluster.sync();
+        cluster_wait();
         St P[2];
 #pragma unroll 1
         for (int q = 0; q < NC; ++q) {
@@ -289,11 +339,15 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
 #pragma unroll
         for (int j = 0; j < 2; ++j)
             S[j] = combine(P[j], sums.get(warp * Cg + col + j), (double)(warp * L) * cc.w2[j]);
+        const int64_t cpair = c0 + col;
+        const int64_t row0 = ((int64_t)b * T + t0 + warp * L) * C + cpair;  // k, v, y offset
+        const bool ok0 = cpair < C, ok1 = cpair + 1 < C;
         if constexpr (kTMA) {
-            // y is staged in place of k (step i reads k_i before writing y_i)
-            auto out_pair = [=](int i, f2 y) { Pair<IO>::store(kr + i * Cg + col, y); };
-            auto out_one = [=](int i, int j, float y) { kr[i * Cg + col + j] = Io<IO>::from_f(y); };
-            chunk_phase3<IO, L>(ref, kr, vr, Cg, col, n, S, cc, out_pair, out_one);
+            // y staged in place of k, sent out by one TMA store of the warp's rows
+            auto st_one = [=](int s, int j, float y) { kr[s * Cg + col + j] = Io<IO>::from_f(y); };
+            auto st_pair = [=](int s, f2 y) { Pair<IO>::store(kr + s * Cg + col, y); };
+            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr, kg + row0, vg + row0, C, ok0, ok1, st_pair,
+                                      st_one);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -303,25 +357,25 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                 }
                 if (round + NB < p.rounds) {
                     bulk_wait_read_all();  // rows free for the next load into this buffer
-                    issue_loads(round + NB);
+                    issue_rows(round + NB);
                 }
             }
             __syncwarp();
         } else {
-            IO* yg = static_cast<IO*>(p.y);
-            const int64_t ybase = ((int64_t)b * T + t0 + warp * L) * C + c0 + col;
-            const int64_t cpair = c0 + col;
-            auto out_one = [=](int i, int j, float y) {
-                if (cpair + j < C) yg[ybase + (int64_t)i * C + j] = Io<IO>::from_f(y);
+            // element-wise stores (any alignment)
+            IO* yrow = yg + row0;
+            auto out_one = [=](int s, int j, float y) {
+                if (j == 0 ? ok0 : ok1) yrow[(int64_t)s * C + j] = Io<IO>::from_f(y);
             };
-            auto out_pair = [=](int i, f2 y) {
-                if (cpair < C) yg[ybase + (int64_t)i * C] = Io<IO>::from_f(lo(y));
-                if (cpair + 1 < C) yg[ybase + (int64_t)i * C + 1] = Io<IO>::from_f(hi(y));
+            auto out_pair = [=](int s, f2 y) {
+                if (ok0) yrow[(int64_t)s * C] = Io<IO>::from_f(lo(y));
+                if (ok1) yrow[(int64_t)s * C + 1] = Io<IO>::from_f(hi(y));
             };
-            chunk_phase3<IO, L>(ref, kr, vr, Cg, col, n, S, cc, out_pair, out_one);
-            __syncwarp();
+            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr, kg + row0, vg + row0, C, ok0, ok1, out_pair,
+                                      out_one);
         }
     }
+    if (kTMA && lane == 0) bulk_wait_read_all();  // staged rows stay valid until read
 
     if (rank == 0 && warp == 0 && p.state_out) {
 #pragma unroll
@@ -330,11 +384,14 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
             if (c < C) store_state_log2(p.state_out, p.BC, (int64_t)b * C + c, carry[j]);
         }
     }
-    if constexpr (kTMA) {
-        if (lane == 0) bulk_wait_read_all();  // the staged rows stay valid until read
-    }
-    // No barrier before leaving: peers only write into this CTA's shared
+    // Every warp's tensor-memory accesses have completed (each load and each
+    // store pass ends in its wait); release the columns.  No cluster barrier
+    // is needed before leaving: peers only write into this CTA's shared
     // memory before a round's cluster barrier, and read only their own.
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    if (warp == 0) tmem_dealloc(tbase, (uint32_t)lay.tmem_cols());
 }
 
 }  // namespace wkv4
