@@ -122,7 +122,8 @@ WKV4_API int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float*
 
 /*
  * Device-side error word of the current device (bit 1: a bounded wait for a
- * TMA copy ran out).  Synchronises the device, reads the word, and clears it
+ * TMA copy ran out; bit 2: a bounded wait for a cluster peer's partial state
+ * ran out).  Synchronises the device, reads the word, and clears it
  * when `reset` is non-zero.  Returns WKV4_OK when the
  * word is zero, WKV4_ERR_TIMEOUT when a wait ran out, WKV4_ERR_CUDA when the
  * read itself failed.

@@ -43,7 +43,8 @@ constexpr float kFastMaxU = 44.f;
 constexpr float kFastMaxW = 0.35f;
 
 // device error word bits
-constexpr unsigned kErrTmaWait = 2u;
+constexpr unsigned kErrTmaWait = 2u;       // a TMA copy did not land in time
+constexpr unsigned kErrExchangeWait = 4u;  // a cluster peer's aggregate did not land in time
 
 
 // A = a 2^p, D = b 2^p.  The max p is carried in fp64 inside the kernels, so
@@ -308,6 +309,49 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------ distributed shared memory
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_u32(uint32_t local_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+    return r;
+}
+
+// Asynchronous stores into (possibly another CTA's) shared memory whose bytes
+// complete a transaction on the mbarrier at `mbar` in the target CTA.
+__device__ __forceinline__ void st_async_v2f32(uint32_t addr, float x, float y, uint32_t mbar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
+        "f"(x), "f"(y), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void st_async_v2f64(uint32_t addr, double x, double y, uint32_t mbar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f64 [%0], {%1, %2}, [%3];" ::"r"(addr),
+        "d"(x), "d"(y), "r"(mbar)
+        : "memory");
+}
+
+// try_wait acquiring at cluster scope (writes by other CTAs' st.async).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitRounds; ++i)
+        if (mbar_try_wait_cluster(bar, parity, 1000000u)) return true;
+    return false;
 }
 
 // ------------------------------------------------ tensor memory (tcgen05)

@@ -13,16 +13,19 @@
 //      go to tensor memory);
 //   2. warp 0 scans the NW chunk summaries (the state contribution before
 //      each chunk, the segment's aggregate) and pushes the aggregate into the
-//      shared memory of every CTA of the cluster (DSMEM stores);
-//   3. one cluster barrier; every warp folds the NC aggregates of the round,
-//      from the state carried into the round, into the state at the segment
-//      start and the state carried into the next round;
+//      shared memory of every CTA of the cluster by asynchronous DSMEM stores
+//      that complete on the receiving CTA's barrier of that round's slot;
+//   3. once all NC aggregates of the round have landed, every warp folds
+//      them, from the state carried into the round, into the state at the
+//      segment start and the state carried into the next round;
 //   4. every warp computes its chunk's outputs from the stash into its k rows
 //      and sends them out with its own TMA store.
 // With several rounds the next round's rows are loaded into a second buffer
 // (NB = 2).
-// There is no global scratch and no spin-wait on another CTA: all exchange is
-// through cluster shared memory and hardware barriers.
+// There is no global scratch: all exchange is through cluster shared memory.
+// Aggregate slots alternate between rounds; a slot's next round's stores
+// come only after every CTA's own push of the round in between, which
+// follows its reads of the slot.  Every wait is bounded.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -33,7 +36,7 @@ namespace wkv4 {
 
 namespace cg = cooperative_groups;
 
-constexpr int kMaxCluster = 8;
+constexpr int kMaxCluster = 8;  // cluster sizes 1, 2, 4, 8; warps per CTA 4 or 8
 
 // Register cap of the scan kernel: two CTAs of 8 warps per SM.
 #ifndef WKV4_SCAN_MAXNREG
@@ -59,8 +62,9 @@ struct ScanLayout {
     __host__ __device__ size_t agg(int slot) const {                                    // [2][nc][Cg] x 16 B
         return params() + (size_t)5 * kCg * 4 + (size_t)slot * nc * kCg * 16;
     }
-    __host__ __device__ size_t bars() const { return agg(2); }  // rows [NB][nw], params x 8 B
-    __host__ __device__ size_t tslot() const { return bars() + (size_t)(NB * nw + 1) * 8; }
+    // rows [NB][nw], params, aggregate slots [2] x 8 B
+    __host__ __device__ size_t bars() const { return agg(2); }
+    __host__ __device__ size_t tslot() const { return bars() + (size_t)(NB * nw + 3) * 8; }
     __host__ __device__ size_t bytes() const { return kAlign + tslot() + 8; }
     // tensor-memory columns: 4 a step for each warp, warps w and w + 4
     // sharing a lane quarter
@@ -105,18 +109,63 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Split cluster barrier: every thread of every CTA of the cluster arrives,
-// then waits.  A releasing arrive publishes this thread's prior stores (the
-// DSMEM pushes) to the threads whose wait acquires; threads with nothing to
-// publish arrive relaxed.
-__device__ __forceinline__ void cluster_arrive_release() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
+// Split cluster barrier (once, at the start): every thread of every CTA of
+// the cluster arrives, then waits.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Warp 0: exclusive prefix of the NW chunk summaries of a segment (in
+// place: entry q becomes the state before chunk q) and the segment aggregate
+// in acc.  All summaries are read before the chain starts; chunk q spans
+// clamp(rem - q L, 0, L) steps.
+template <int NW, int L>
+__device__ __forceinline__ void scan_chunks(const TripleRef& sums, int col, int rem,
+                                            const PairConsts& cc, St (&acc)[2]) {
+    constexpr int Cg = 64;
+    St x[NW][2];
+#pragma unroll
+    for (int q = 0; q < NW; ++q)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) x[q][j] = sums.get(q * Cg + col + j);
+    acc[0] = acc[1] = empty_state();
+#pragma unroll
+    for (int q = 0; q < NW; ++q) {
+        const double nq = (double)max(0, min(L, rem - q * L));
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            sums.put(q * Cg + col + j, acc[j]);
+            acc[j] = combine(acc[j], x[q][j], nq * cc.w2[j]);
+        }
+    }
+}
+
+// Every warp: fold of the NC segment aggregates of a round into the state at
+// this CTA's segment start (P) and the state carried into the next round
+// (carry); segment q spans clamp(rrem - q Ts, 0, Ts) steps.
+template <int NC>
+__device__ __forceinline__ void fold_aggs(const TripleRef& agg, int col, int rank, int64_t rrem,
+                                          int Ts, const PairConsts& cc, St (&carry)[2], St (&P)[2]) {
+    constexpr int Cg = 64;
+    St y[NC][2];
+#pragma unroll
+    for (int q = 0; q < NC; ++q)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) y[q][j] = agg.get(q * Cg + col + j);
+    P[0] = carry[0];
+    P[1] = carry[1];
+#pragma unroll
+    for (int q = 0; q < NC; ++q) {
+        const double nq = (double)max((int64_t)0, min((int64_t)Ts, rrem - (int64_t)q * Ts));
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            if (q == rank) P[j] = carry[j];
+            carry[j] = combine(carry[j], y[q][j], nq * cc.w2[j]);
+        }
+    }
 }
 
 template <typename IO, int L, int NB, bool kTMA>
@@ -139,6 +188,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     const TripleRef sums = triples(base + lay.sums(), NW * Cg);       // [NW][Cg]
     uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // rows [NB][NW], params
     uint64_t* pbar = mbar + NB * NW;
+    uint64_t* abar = pbar + 1;  // [2]: the aggregates of a round have landed
     uint32_t* tslot = reinterpret_cast<uint32_t*>(base + lay.tslot());
     float* sw = reinterpret_cast<float*>(base + lay.params());  // [5][Cg]: w, u, a, b, p
 
@@ -183,7 +233,15 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     // with aligned pointers comes by bulk copy on its own mbarrier, issued
     // before the rows, so it does not queue behind other CTAs' row traffic.
     const bool bulk = kTMA && p.bulk_params && c0 + Cg <= C;
+    // every CTA of the cluster pushes 32 B per lane into each aggregate slot
+    const uint32_t agg_bytes = (uint32_t)NC * 32u * 32u;
     if (warp == 0) tmem_alloc(tslot, (uint32_t)lay.tmem_cols());
+    if (threadIdx.x == 0) {
+        mbar_init(abar, 1);
+        mbar_init(abar + 1, 1);
+        fence_mbar_init();
+        for (int r = 0; r < 2 && r < p.rounds; ++r) mbar_arrive_expect_tx(abar + r, agg_bytes);
+    }
     if constexpr (kTMA) {
         if (lane == 0) {
             if (warp == 0) {
@@ -225,8 +283,9 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     tmem_fence_before_sync();
     __syncthreads();
     tmem_fence_after_sync();
-    // the CTAs of the cluster have all started before the first DSMEM store
-    // (this barrier's wait comes just before it)
+    // the CTAs of the cluster have all started, with their barriers
+    // initialised, before the first DSMEM store (this barrier's wait comes
+    // just before it)
     cluster_arrive_relaxed();
     const uint32_t tbase = *tslot;
     // this warp's stash: its lane quarter, 4 L columns for each warp of the quarter
@@ -286,51 +345,50 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         __syncthreads();
 
         // ---- 2. warp 0: exclusive prefix of the chunk summaries (in place); the
-        //         segment aggregate is pushed into slot [round & 1][rank] of every
-        //         CTA of the cluster
+        //         segment aggregate goes by asynchronous DSMEM stores into slot
+        //         [round & 1][rank] of every CTA of the cluster, each store
+        //         completing bytes on that CTA's barrier of the slot
         const int slot = round & 1;
         const TripleRef agg = triples(base + lay.agg(slot), NC * Cg);
+        // steps of this CTA's segment (the chunks' lengths follow from it)
+        const int rem = (int)max((int64_t)0, min((int64_t)Ts, T - t0));
         if (round == 0) cluster_wait();  // every CTA of the cluster has started
         if (warp == 0) {
-            St acc[2] = {empty_state(), empty_state()};
-#pragma unroll 1
-            for (int q = 0; q < NW; ++q) {
-                const double nq = (double)chunk_len(round, q);
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int i = q * Cg + col + j;
-                    const St Sq = sums.get(i);
-                    sums.put(i, acc[j]);
-                    acc[j] = combine(acc[j], Sq, nq * cc.w2[j]);
-                }
+            St acc[2];
+            if (NW == 8) {
+                scan_chunks<8, L>(sums, col, rem, cc, acc);
+            } else {
+                scan_chunks<4, L>(sums, col, rem, cc, acc);
             }
             const int off = rank * Cg + col;
+            const uint32_t la = smem_u32(agg.a + off), lb = smem_u32(agg.b + off);
+            const uint32_t lp = smem_u32(agg.p + off), lbar = smem_u32(abar + slot);
 #pragma unroll 1
             for (int q = 0; q < NC; ++q) {
-                float* ra = cluster.map_shared_rank(agg.a, q);
-                float* rb = cluster.map_shared_rank(agg.b, q);
-                double* rp = cluster.map_shared_rank(agg.p, q);
-                *reinterpret_cast<float2*>(ra + off) = make_float2(acc[0].a, acc[1].a);
-                *reinterpret_cast<float2*>(rb + off) = make_float2(acc[0].b, acc[1].b);
-                rp[off] = acc[0].p;
-                rp[off + 1] = acc[1].p;
+                const uint32_t rbar = mapa_u32(lbar, (uint32_t)q);
+                st_async_v2f32(mapa_u32(la, (uint32_t)q), acc[0].a, acc[1].a, rbar);
+                st_async_v2f32(mapa_u32(lb, (uint32_t)q), acc[0].b, acc[1].b, rbar);
+                st_async_v2f64(mapa_u32(lp, (uint32_t)q), acc[0].p, acc[1].p, rbar);
             }
-            cluster_arrive_release();
-        } else {
-            cluster_arrive_relaxed();
         }
+        __syncthreads();  // the exclusive prefixes are in place
 
-        // ---- 3. every warp folds the round's aggregates from its own shared memory
-        cluster_wait();
+        // ---- 3. every warp folds the round's aggregates once they have landed
+        if (!failed && !mbar_wait_cluster_bounded(abar + slot, (uint32_t)((round >> 1) & 1))) {
+            failed = true;
+            if (lane == 0) atomicOr(&g_device_error, kErrExchangeWait);
+        }
+        // the slot's next use is round + 2: its pushes follow this CTA's own
+        // push of round + 1, so the barrier is re-armed well before them
+        if (threadIdx.x == 0 && round + 2 < p.rounds) mbar_arrive_expect_tx(abar + slot, agg_bytes);
         St P[2];
-#pragma unroll 1
-        for (int q = 0; q < NC; ++q) {
-            const int64_t sq = t0 + (int64_t)(q - rank) * Ts;
-            const double nq = (double)max((int64_t)0, min((int64_t)Ts, T - sq));
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                if (q == rank) P[j] = carry[j];
-                carry[j] = combine(carry[j], agg.get(q * Cg + col + j), nq * cc.w2[j]);
+        {
+            const int64_t rrem = T - (t0 - (int64_t)rank * Ts);  // steps of the round from segment 0 on
+            switch (NC) {
+                case 1: fold_aggs<1>(agg, col, rank, rrem, Ts, cc, carry, P); break;
+                case 2: fold_aggs<2>(agg, col, rank, rrem, Ts, cc, carry, P); break;
+                case 4: fold_aggs<4>(agg, col, rank, rrem, Ts, cc, carry, P); break;
+                default: fold_aggs<8>(agg, col, rank, rrem, Ts, cc, carry, P); break;
             }
         }
 
