@@ -57,7 +57,13 @@ struct ScanLayout {
     __host__ __device__ size_t tile() const { return (size_t)nw * kChunkBytes; }
     __host__ __device__ size_t k(int buf) const { return (size_t)buf * 2 * tile(); }
     __host__ __device__ size_t v(int buf) const { return k(buf) + tile(); }
-    __host__ __device__ size_t sums() const { return (size_t)NB * 2 * tile(); }          // [nw][Cg] x 16 B
+    // y staging: in place of k with one round, its own tile with several (so
+    // that the rows take the next load as soon as the summary pass is done)
+    static constexpr bool kOwnY = NB > 1;
+    __host__ __device__ size_t ys() const { return kOwnY ? (size_t)NB * 2 * tile() : k(0); }
+    __host__ __device__ size_t sums() const {  // [nw][Cg] x 16 B
+        return (size_t)NB * 2 * tile() + (kOwnY ? tile() : 0);
+    }
     __host__ __device__ size_t params() const { return sums() + (size_t)nw * kCg * 16; }  // [5][Cg] f32
     __host__ __device__ size_t agg(int slot) const {                                    // [2][nc][Cg] x 16 B
         return params() + (size_t)5 * kCg * 4 + (size_t)slot * nc * kCg * 16;
@@ -209,6 +215,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         return (int)max((int64_t)0, min((int64_t)L, T - tc));
     };
     auto rows_k = [&](int buf) { return reinterpret_cast<IO*>(base + lay.k(buf)) + warp * L * Cg; };
+    IO* const ystage = reinterpret_cast<IO*>(base + lay.ys()) + warp * L * Cg;  // with kOwnY
     auto rows_v = [&](int buf) { return reinterpret_cast<IO*>(base + lay.v(buf)) + warp * L * Cg; };
     // Lane 0 of each warp: this warp's rows of round j into buffer j % NB.
     // Every round completes one phase of the warp's barrier of that buffer (a
@@ -342,6 +349,10 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         chunk_phase1<IO, L, true>(ref, kr, vr, Cg, col, n, cc, sum, taddr);
 #pragma unroll
         for (int j = 0; j < 2; ++j) sums.put(warp * Cg + col + j, sum[j]);
+        if constexpr (kTMA && Lay::kOwnY) {
+            __syncwarp();  // every lane has read the rows: they take round + NB's
+            if (lane == 0) issue_rows(round + NB);
+        }
         __syncthreads();
 
         // ---- 2. warp 0: exclusive prefix of the chunk summaries (in place); the
@@ -401,21 +412,23 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         const int64_t row0 = ((int64_t)b * T + t0 + warp * L) * C + cpair;  // k, v, y offset
         const bool ok0 = cpair < C, ok1 = cpair + 1 < C;
         if constexpr (kTMA) {
-            // y staged in place of k, sent out by one TMA store of the warp's rows
-            auto st_one = [=](int s, int j, float y) { kr[s * Cg + col + j] = Io<IO>::from_f(y); };
-            auto st_pair = [=](int s, f2 y) { Pair<IO>::store(kr + s * Cg + col, y); };
+            // y staged (in place of k, or in the staging tile once the previous
+            // round's store has read it), sent out by one TMA store
+            IO* yr = Lay::kOwnY ? ystage : kr;
+            if (Lay::kOwnY && round > 0) {
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+            }
+            auto st_one = [=](int s, int j, float y) { yr[s * Cg + col + j] = Io<IO>::from_f(y); };
+            auto st_pair = [=](int s, f2 y) { Pair<IO>::store(yr + s * Cg + col, y); };
             chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr, kg + row0, vg + row0, C, ok0, ok1, st_pair,
                                       st_one);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 if (n > 0 && !failed) {
-                    tma_store_3d(&tmy, kr, (int)c0, (int)(t0 + warp * L), b);
+                    tma_store_3d(&tmy, yr, (int)c0, (int)(t0 + warp * L), b);
                     bulk_commit();
-                }
-                if (round + NB < p.rounds) {
-                    bulk_wait_read_all();  // rows free for the next load into this buffer
-                    issue_rows(round + NB);
                 }
             }
             __syncwarp();
