@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="run the workload's shape with this T instead (small profiling captures; "
+                         "the line then names the shape it ran)")
     return ap.parse_args()
 
 
@@ -220,7 +223,7 @@ def run_native(args):
     torch.cuda.set_device(dev)
     wkv4.load()
     variant = VARIANTS[args.variant]
-    wl = synth.workload(args.workload)
+    wl = synth.workload(args.workload, **({"T": args.seq_len} if args.seq_len else {}))
     x = synth.forward_inputs(wl.replace(seed=wl.seed + 1000 * rank) if rank else wl)
 
     per_set = 2 * io_bytes(wl) + io_bytes(wl) + 24 * wl.B * wl.C
