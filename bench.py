@@ -15,6 +15,13 @@ the region (CUDA events on the launching stream) is max-reduced over ranks.
 Under torchrun each rank processes its own batch (independent sequences, no
 collective on the data path): weak scaling.
 
+A decode workload (T = 1, e.g. ``--workload decode_b256``: B=256, C=5120,
+bf16, 1024 calls) times the batched decode instead: one step is the whole
+loop of wkv4_decode_step calls over one fp32 state updated in place, captured
+as one CUDA graph; each call's k, v come from a pool of seeded inputs that
+rotates over more than 3x the L2 cache.  The state (12 B a channel) stays
+L2-resident across calls by design, so the line's GB/s is effective.
+
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead
 (rank 0 only; other ranks exit).
 """
@@ -43,8 +50,10 @@ VARIANTS = {"auto": 0, "seq": 1, "scan": 2, "scan_ldg": 3, "step": 4}
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 20000 calls; 20 loops for a decode workload)")
+    ap.add_argument("--warmup", type=int, default=None,
+                    help="untimed steps (default 200 calls; 3 loops for a decode workload)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="rwkv4_169m_prefill")
     ap.add_argument("--variant", default="auto", choices=sorted(VARIANTS))
@@ -385,7 +394,14 @@ def run_reference(args):
     from rwkv_wkv_linear_b200 import synth
 
     wl = synth.workload(args.workload)
-    x = synth.forward_inputs(wl)
+    config = {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C, "io_dtype": wl.dtype}
+    if wl.T == 1:
+        # a decode loop over one state is a forward over the calls' time axis
+        wl, x = _decode_as_forward(wl)
+        config.update(calls=synth.workload(args.workload).steps,
+                      sampled_as=f"forward B={wl.B}, T={wl.T} (batch rows x calls)")
+    else:
+        x = synth.forward_inputs(wl)
     cores = len(os.sched_getaffinity(0))
     BC = wl.B * wl.C
     # calibrate: channel-steps per second of the oracle on this host
@@ -411,7 +427,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C, "io_dtype": wl.dtype},
+        "config": config,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -436,10 +452,203 @@ def _ref_sample(x, wl, n_ch):
     return (np.ascontiguousarray(k[None]), np.ascontiguousarray(v[None]), w, u, s)
 
 
+def run_decode(args):
+    """Batched decode: K loops of wl.steps wkv4_decode_step calls (one CUDA
+    graph per loop) over one state; the device time of the K loops."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from rwkv_wkv_linear_b200 import synth, wkv4
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wkv4.load()
+    wl = synth.workload(args.workload)
+    if rank:
+        wl = wl.replace(seed=wl.seed + 1000 * rank)
+    w, u = (t.to(dev) for t in synth.decode_params(wl))
+    call_io = 2 * io_bytes(wl)  # k, v of one call
+    pool = max(8, -(-3 * L2_BYTES // call_io))
+    ks, vs = [], []
+    for s_ in range(pool):
+        k, v = synth.decode_step_inputs(wl, s_)
+        ks.append(k.to(dev))
+        vs.append(v.to(dev))
+    ys = [torch.empty_like(ks[0]) for _ in range(pool)]
+    state = synth.zero_state(wl.B, wl.C).to(dev)
+    stream = torch.cuda.Stream(device=dev)
+    n = wl.steps
+
+    def loop():
+        for s_ in range(n):
+            j = s_ % pool
+            wkv4.decode_step(ks[j], vs[j], w, u, state, y=ys[j], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            loop()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        loop()
+    with torch.cuda.stream(stream):
+        g.replay()  # upload (untimed)
+    stream.synchronize()
+
+    K = args.steps
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
+    clocks.start()
+    time.sleep(0.2)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(K):
+            g.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    ms = max_over_ranks(start.elapsed_time(end), dev)
+    if wkv4.device_error() != 0:
+        raise RuntimeError("device-side wait ran out during the timed region")
+
+    # end to end through the C ABI: every call's k, v from pinned host memory,
+    # its y back to the host
+    e2e = None
+    if not args.no_e2e:
+        n_e2e = max(1, args.e2e_steps)
+        kh = [ks[j % pool].cpu().pin_memory() for j in range(min(pool, n_e2e))]
+        vh = [vs[j % pool].cpu().pin_memory() for j in range(min(pool, n_e2e))]
+        yh = torch.empty_like(kh[0]).pin_memory()
+        kd, vd, yd = ks[0], vs[0], ys[0]
+
+        def e2e_call(j):
+            kd.copy_(kh[j % len(kh)], non_blocking=True)
+            vd.copy_(vh[j % len(vh)], non_blocking=True)
+            wkv4.decode_step(kd, vd, w, u, state, y=yd, stream=stream)
+            yh.copy_(yd, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for j in range(3):
+                e2e_call(j)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        with torch.cuda.stream(stream):
+            for j in range(n_e2e):
+                e2e_call(j)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        t2_ms = max_over_ranks(s2.elapsed_time(e2), dev)
+        e2e = {"value": job_throughput(wl.B * wl.C, n_e2e, world, t2_ms), "unit": UNIT,
+               "h2d_bytes_per_step": call_io, "d2h_bytes_per_step": io_bytes(wl),
+               "steps": n_e2e, "step": "one decode call"}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        calls = K * n
+        call_bytes = 3 * io_bytes(wl) + 24 * wl.B * wl.C  # k, v, y + state read and written
+        achieved = call_bytes / (ms / 1e3 / calls) / 1e9
+        line = {
+            "metric": METRIC,
+            "value": job_throughput(wl.channel_steps, K, world, ms),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms / K,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C, "calls": n,
+                       "io_dtype": wl.dtype, "state": "fp32, in place, zero at the start",
+                       "global_batch": wl.B * world, "seq_len": n,
+                       "parallelism": f"independent sequences per rank (x{world})",
+                       "step": f"one decode loop of {n} wkv4_decode_step calls",
+                       "l2": f"k, v rotate over {pool} seeded call inputs "
+                             f"({pool * call_io / 1e6:.0f} MB > 3x L2); the state is L2-resident",
+                       "launch": f"one CUDA graph of {n} calls per step, {K} replays"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "bytes_per_launch": call_bytes, "effective": True,
+                         "traffic": recorded_traffic(wl.name, "auto")},
+            "gpu_launches": calls,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_decode(wl)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _decode_as_forward(wl, rows: int = 16, calls: int = 128):
+    """The first `rows` batch rows and `calls` calls of a decode workload as
+    forward inputs (B = rows, T = calls), with its w, u and the zero state."""
+    import torch
+    from rwkv_wkv_linear_b200 import synth
+    w, u = synth.decode_params(wl)
+    calls = min(calls, wl.steps)
+    ks, vs = [], []
+    for s_ in range(calls):
+        k, v = synth.decode_step_inputs(wl, s_)
+        ks.append(k[:rows])
+        vs.append(v[:rows])
+    x = {"w": w, "u": u, "k": torch.stack(ks, dim=1), "v": torch.stack(vs, dim=1),
+         "state_in": None}
+    return wl.replace(name=wl.name, B=min(rows, wl.B), T=calls, steps=1), x
+
+
+def cpu_baseline_decode(wl):
+    """The oracle over a bounded sample of the decode workload (see
+    _decode_as_forward)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    ws, x = _decode_as_forward(wl)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward(x["k"], x["v"], x["w"], x["u"], None, nthreads=cores)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if reps >= 3 and dt > 1.0 or dt > 20.0:
+            break
+    return {"value": ws.channel_steps * reps / dt / 1e9, "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"batch rows 0..{ws.B - 1} of {wl.B} x calls 0..{ws.T - 1} of {wl.steps}, "
+                      f"C={wl.C} ({ws.channel_steps} channel-steps) x {reps} passes, fp64 C "
+                      f"recurrence, {cores} threads over channels"}
+
+
 def main():
     args = parse()
+    from rwkv_wkv_linear_b200 import synth
+    decode = synth.workload(args.workload).T == 1
+    if args.steps is None:
+        args.steps = 20 if decode else 20000
+    if args.warmup is None:
+        args.warmup = 3 if decode else 200
     if args.impl == "reference":
         run_reference(args)
+    elif decode:
+        run_decode(args)
     else:
         run_native(args)
 

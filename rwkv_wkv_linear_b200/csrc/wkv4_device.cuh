@@ -111,18 +111,24 @@ __device__ __forceinline__ void exact_update(St& s, float k, float v, double w2)
 // The per-step max-trick with the state in natural units (the units of the
 // state buffers), fp64 max and accurate exp2f: the decode step and the
 // per-step kernel, where one step's rounding is carried to the next call.
+// Of the two scale factors of each half step the one at the max is exactly
+// 1 (exp2f(0)), so only the other one is evaluated: the same bits as taking
+// both, with half the exponentials.
 __device__ __forceinline__ float step_nat(St& s, float k, float v, float w, float u) {
     const double kd = k;
-    const double q = fmax(s.p, (double)u + kd);
-    const float f1 = exp2f((float)(s.p - q) * kLog2e);
-    const float f2 = exp2f((float)((double)u + kd - q) * kLog2e);
+    // output: q = max(p, u + k)
+    const double d1 = s.p - ((double)u + kd);
+    const float f = exp2f((float)-fabs(d1) * kLog2e);
+    const float f1 = d1 >= 0.0 ? 1.f : f, f2 = d1 >= 0.0 ? f : 1.f;
     const float y = __fdividef(fmaf(f1, s.a, f2 * v), fmaf(f1, s.b, f2));
-    const double q2 = fmax(s.p + (double)w, kd);
-    const float g1 = exp2f((float)(s.p + (double)w - q2) * kLog2e);
-    const float g2 = exp2f((float)(kd - q2) * kLog2e);
+    // state: q2 = max(p + w, k)
+    const double pw = s.p + (double)w;
+    const double d2 = pw - kd;
+    const float g = exp2f((float)-fabs(d2) * kLog2e);
+    const float g1 = d2 >= 0.0 ? 1.f : g, g2 = d2 >= 0.0 ? g : 1.f;
     s.a = fmaf(g1, s.a, g2 * v);
     s.b = fmaf(g1, s.b, g2);
-    s.p = q2;
+    s.p = d2 >= 0.0 ? pw : kd;
     return y;
 }
 
