@@ -402,10 +402,15 @@ __device__ __noinline__ void chunk_exact_global(const IO* gk, const IO* gv, int6
 // Outputs of a chunk of n steps whose summary pass left its stash in tensor
 // memory at taddr (chunk_phase1 with kStash).  When every lane of the warp
 // has both channels on the fixed-reference path (the decision is warp-wide:
-// tensor-memory loads are warp-collective), from the state (alpha, beta) at
-// the chunk start rescaled to the reference,
-//   y_i = (e^{i w} alpha + N_i) / (e^{i w} beta + Dn_i),
-// one reciprocal a step, through out_pair(i, y); otherwise the exact per-step
+// tensor-memory loads are warp-collective), from the state S = (a, b, p) at
+// the chunk start, whose weight at step i relative to the reference r is
+// f_i = 2^{p - r} e^{i w},
+//   y_i = (f_i a + N_i) / (f_i b + Dn_i),
+// one reciprocal a step, through out_pair(i, y).  f_i is carried as one
+// factor (f_0 = 2^{p - r}, times e^w a step), so it leaves the float range
+// only where the state's share of y_i does: a separate e^{i w} would
+// underflow under a fast decay while the state, lifted up to 2^63 above the
+// reference, still outweighs Dn_i.  Otherwise the exact per-step
 // path from k, v in global memory (gk, gv: the pair's first channel at the
 // chunk's first step, row stride `stride`; ok[j]: channel j exists) through
 // out_one(i, j, y).
@@ -418,18 +423,16 @@ __device__ __forceinline__ void chunk_phase3_stash(const PairRef& r, int n, cons
     static_assert(L % 4 == 0, "stash: whole column groups");
     if (n <= 0) return;
     bool f3[2];
-    float a0[2], b0[2];
+    float sc[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         const double lift = S[j].p - (double)r.kref[j];
         f3[j] = r.fast[j] && (lift <= (double)(kFastStateLift * kLog2e));
-        const float sc = ex2((float)lift);
-        a0[j] = S[j].a * sc;
-        b0[j] = S[j].b * sc;
+        sc[j] = ex2((float)lift);
     }
     if (__all_sync(0xffffffffu, f3[0] && f3[1])) {
-        const f2 al = pk(a0[0], a0[1]), be = pk(b0[0], b0[1]);
-        f2 f = pk(1.f, 1.f);  // e^{i w}
+        const f2 al = pk(S[0].a, S[1].a), be = pk(S[0].b, S[1].b);
+        f2 f = pk(sc[0], sc[1]);  // 2^{p - r} e^{i w}
         if (n == L) {
 #pragma unroll
             for (int q = 0; q < L / 4; ++q) {

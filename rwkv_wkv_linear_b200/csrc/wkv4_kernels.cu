@@ -121,11 +121,11 @@ struct ScanOcc {
     std::atomic<int> bps[64][2];
 };
 
-template <typename IO, int L, int NB, bool kTMA>
+template <typename IO, int L, bool kMulti, bool kTMA>
 static cudaError_t scan_occupancy(int (&bps)[2]) {
     static DeviceFlags attr;
     static ScanOcc occ;
-    auto kern = wkv4_scan_kernel<IO, L, NB, kTMA>;
+    auto kern = wkv4_scan_kernel<IO, L, kMulti, kTMA>;
     cudaError_t e = ensure_smem_attr(attr, kern, kMaxSmem);
     if (e != cudaSuccess) return e;
     int dev = 0;
@@ -136,7 +136,7 @@ static cudaError_t scan_occupancy(int (&bps)[2]) {
         if (v == 0) {
             v = -1;
             // the largest cluster's layout: a bound for every cluster size
-            const ScanLayout<IO, L, NB> lay{kNwChoices[i], kMaxCluster};
+            const ScanLayout<IO, L, kMulti> lay{kNwChoices[i], kMaxCluster};
             const size_t req = scan_smem_request(lay.bytes(), lay.tmem_cols());
             if (req <= kMaxSmem) {
                 int n = 0;
@@ -159,15 +159,15 @@ static cudaError_t scan_occupancy(int (&bps)[2]) {
 // whose grid still fits in one wave (a second wave of CTAs that each walk all
 // of T would be costly).  WKV4_SCAN_NW / WKV4_SCAN_CLUSTER override (tuning).
 struct ScanShape {
-    int nw, nc, rounds, nb;
+    int nw, nc, rounds;
 };
 
 template <typename IO, int L, bool kTMA>
 static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
-    int b1[2], b2[2];
-    cudaError_t e = scan_occupancy<IO, L, 1, kTMA>(b1);
+    int b1[2], b2[2];  // one round, several rounds
+    cudaError_t e = scan_occupancy<IO, L, false, kTMA>(b1);
     if (e != cudaSuccess) return e;
-    if ((e = scan_occupancy<IO, L, 2, kTMA>(b2)) != cudaSuccess) return e;
+    if ((e = scan_occupancy<IO, L, true, kTMA>(b2)) != cudaSuccess) return e;
     const int sms = sm_count();
     const int force_nw = env_int("WKV4_SCAN_NW", 0), force_nc = env_int("WKV4_SCAN_CLUSTER", 0);
     for (int i = 0; i < 2; ++i) {
@@ -185,15 +185,14 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
         }
         const int64_t rounds = (nseg + nc - 1) / nc;
         if (rounds > (1ll << 30)) continue;
-        const int nb = (kTMA && rounds > 1) ? 2 : 1;
-        if ((nb == 1 ? b1[i] : b2[i]) <= 0) continue;  // does not fit on an SM
-        out = {nw, nc, (int)rounds, nb};
+        if ((rounds == 1 ? b1[i] : b2[i]) <= 0) continue;  // does not fit on an SM
+        out = {nw, nc, (int)rounds};
         return cudaSuccess;
     }
     return cudaErrorInvalidConfiguration;
 }
 
-template <typename IO, int L, int NB, bool kTMA>
+template <typename IO, int L, bool kMulti, bool kTMA>
 static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const ScanShape& sh,
                                   int64_t tiles, EncodeFn encode) {
     CUtensorMap tk, tv, ty;
@@ -206,8 +205,8 @@ static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const S
             !encode(&ty, a.y, a.dtype, a.B, a.T, a.C, 64, L))
             return cudaErrorInvalidValue;
     }
-    auto kern = wkv4_scan_kernel<IO, L, NB, kTMA>;
-    const ScanLayout<IO, L, NB> lay{sh.nw, sh.nc};
+    auto kern = wkv4_scan_kernel<IO, L, kMulti, kTMA>;
+    const ScanLayout<IO, L, kMulti> lay{sh.nw, sh.nc};
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(tiles * sh.nc), 1, 1);
@@ -247,8 +246,8 @@ static cudaError_t launch_scan_t(const FwdArgs& a, EncodeFn encode) {
     if (e != cudaSuccess) return e;
     if (tiles * sh.nc > (int64_t)INT32_MAX) return cudaErrorInvalidConfiguration;
     p.rounds = sh.rounds;
-    if (sh.nb == 1) return launch_scan_nb<IO, L, 1, kTMA>(a, p, sh, tiles, encode);
-    return launch_scan_nb<IO, L, 2, kTMA>(a, p, sh, tiles, encode);
+    if (sh.rounds == 1) return launch_scan_nb<IO, L, false, kTMA>(a, p, sh, tiles, encode);
+    return launch_scan_nb<IO, L, true, kTMA>(a, p, sh, tiles, encode);
 }
 
 cudaError_t launch_scan(const FwdArgs& a, bool tma, EncodeFn encode) {

@@ -18,14 +18,16 @@
 //   3. once all NC aggregates of the round have landed, every warp folds
 //      them, from the state carried into the round, into the state at the
 //      segment start and the state carried into the next round;
-//   4. every warp computes its chunk's outputs from the stash into its k rows
-//      and sends them out with its own TMA store.
-// With several rounds the next round's rows are loaded into a second buffer
-// (NB = 2).
-// There is no global scratch: all exchange is through cluster shared memory.
-// Aggregate slots alternate between rounds; a slot's next round's stores
-// come only after every CTA's own push of the round in between, which
-// follows its reads of the slot.  Every wait is bounded.
+//   4. every warp computes its chunk's outputs from the stash.
+// One round: y is staged in the warp's k rows and sent out by one TMA store.
+// Several rounds (kMulti) are software-pipelined: a warp's rows take the next
+// round's load right after its summary pass; round r + 1's summary pass runs
+// before round r's steps 3 and 4, and warp 0 scans and pushes round r + 1
+// right after its step 4 of round r, so the aggregates travel while the
+// other warps work.  The chunk summaries and the stash alternate between two
+// slots, the aggregates rotate through three; y goes straight from registers
+// to global memory.  There is no global scratch: all exchange is through
+// cluster shared memory.  Every wait is bounded.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -44,37 +46,37 @@ constexpr int kMaxCluster = 8;  // cluster sizes 1, 2, 4, 8; warps per CTA 4 or 
 #endif
 
 // Shared-memory layout for nw warps and clusters of nc (offsets from a
-// 128-byte aligned base): NB row buffers of k and v, the chunk summaries,
-// the tile's w, u and state, barriers, two slots of aggregates.
-template <typename IO, int L, int NB>
+// 128-byte aligned base): one buffer of k and v rows, the chunk summaries,
+// the tile's w, u and state, barriers, the aggregate slots.  kMulti (T walked
+// in several rounds, software-pipelined): two slots of chunk summaries and of
+// the stash, three of aggregates.
+template <typename IO, int L, bool kMulti>
 struct ScanLayout {
     static constexpr int kCg = 64;  // channels per tile: 32 lanes x 2
     static constexpr int kChunkBytes = L * kCg * (int)sizeof(IO);  // one warp's rows, one tensor
     static constexpr int kAlign = 128;                               // TMA destinations
+    static constexpr int kSlots = kMulti ? 2 : 1;                    // summaries, stash
+    static constexpr int kAggSlots = kMulti ? 3 : 1;
     static_assert(L <= 256 && L % 4 == 0, "TMA box dims, stash column groups");
     static_assert(kChunkBytes % kAlign == 0, "TMA destination alignment");
     int nw, nc;
     __host__ __device__ size_t tile() const { return (size_t)nw * kChunkBytes; }
-    __host__ __device__ size_t k(int buf) const { return (size_t)buf * 2 * tile(); }
-    __host__ __device__ size_t v(int buf) const { return k(buf) + tile(); }
-    // y staging: in place of k with one round, its own tile with several (so
-    // that the rows take the next load as soon as the summary pass is done)
-    static constexpr bool kOwnY = NB > 1;
-    __host__ __device__ size_t ys() const { return kOwnY ? (size_t)NB * 2 * tile() : k(0); }
-    __host__ __device__ size_t sums() const {  // [nw][Cg] x 16 B
-        return (size_t)NB * 2 * tile() + (kOwnY ? tile() : 0);
+    __host__ __device__ size_t k() const { return 0; }
+    __host__ __device__ size_t v() const { return tile(); }
+    __host__ __device__ size_t sums(int slot) const {  // [kSlots][nw][Cg] x 16 B
+        return 2 * tile() + (size_t)slot * nw * kCg * 16;
     }
-    __host__ __device__ size_t params() const { return sums() + (size_t)nw * kCg * 16; }  // [5][Cg] f32
-    __host__ __device__ size_t agg(int slot) const {                                    // [2][nc][Cg] x 16 B
+    __host__ __device__ size_t params() const { return sums(kSlots); }  // [5][Cg] f32
+    __host__ __device__ size_t agg(int slot) const {                    // [kAggSlots][nc][Cg] x 16 B
         return params() + (size_t)5 * kCg * 4 + (size_t)slot * nc * kCg * 16;
     }
-    // rows [NB][nw], params, aggregate slots [2] x 8 B
-    __host__ __device__ size_t bars() const { return agg(2); }
-    __host__ __device__ size_t tslot() const { return bars() + (size_t)(NB * nw + 3) * 8; }
+    // rows [nw], params, aggregate slots [kAggSlots] x 8 B
+    __host__ __device__ size_t bars() const { return agg(kAggSlots); }
+    __host__ __device__ size_t tslot() const { return bars() + (size_t)(nw + 1 + kAggSlots) * 8; }
     __host__ __device__ size_t bytes() const { return kAlign + tslot() + 8; }
-    // tensor-memory columns: 4 a step for each warp, warps w and w + 4
-    // sharing a lane quarter
-    __host__ __device__ int tmem_cols() const { return nw * L; }
+    // tensor-memory columns: 4 a step for each warp and slot, warps w and
+    // w + 4 sharing a lane quarter
+    __host__ __device__ int tmem_cols() const { return kSlots * nw * L; }
 };
 
 struct ScanParams {
@@ -174,11 +176,12 @@ __device__ __forceinline__ void fold_aggs(const TripleRef& agg, int col, int ran
     }
 }
 
-template <typename IO, int L, int NB, bool kTMA>
+template <typename IO, int L, bool kMulti, bool kTMA>
 __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     wkv4_scan_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __grid_constant__ CUtensorMap tmy, const ScanParams p) {
-    using Lay = ScanLayout<IO, L, NB>;
+    using Lay = ScanLayout<IO, L, kMulti>;
+    constexpr int kAS = Lay::kAggSlots;
     constexpr int Cg = Lay::kCg;
     constexpr int kChunkBytes = Lay::kChunkBytes;
     constexpr unsigned kAlign = Lay::kAlign;
@@ -191,10 +194,9 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     // align by offsetting the shared array itself (a round trip through an
     // integer would lose the address space and turn every access generic)
     unsigned char* base = smem_raw + ((kAlign - (smem_u32(smem_raw) & (kAlign - 1))) & (kAlign - 1));
-    const TripleRef sums = triples(base + lay.sums(), NW * Cg);       // [NW][Cg]
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // rows [NB][NW], params
-    uint64_t* pbar = mbar + NB * NW;
-    uint64_t* abar = pbar + 1;  // [2]: the aggregates of a round have landed
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // rows [NW], params
+    uint64_t* pbar = mbar + NW;
+    uint64_t* abar = pbar + 1;  // [kAS]: the aggregates of a round have landed
     uint32_t* tslot = reinterpret_cast<uint32_t*>(base + lay.tslot());
     float* sw = reinterpret_cast<float*>(base + lay.params());  // [5][Cg]: w, u, a, b, p
 
@@ -214,22 +216,20 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         const int64_t tc = (int64_t)j * seg_stride + (int64_t)rank * Ts + (int64_t)q * L;
         return (int)max((int64_t)0, min((int64_t)L, T - tc));
     };
-    auto rows_k = [&](int buf) { return reinterpret_cast<IO*>(base + lay.k(buf)) + warp * L * Cg; };
-    IO* const ystage = reinterpret_cast<IO*>(base + lay.ys()) + warp * L * Cg;  // with kOwnY
-    auto rows_v = [&](int buf) { return reinterpret_cast<IO*>(base + lay.v(buf)) + warp * L * Cg; };
-    // Lane 0 of each warp: this warp's rows of round j into buffer j % NB.
-    // Every round completes one phase of the warp's barrier of that buffer (a
-    // plain arrive where nothing is copied), so its phases stay in step.
+    IO* const kr = reinterpret_cast<IO*>(base + lay.k()) + warp * L * Cg;  // this warp's rows
+    IO* const vr = reinterpret_cast<IO*>(base + lay.v()) + warp * L * Cg;
+    // Lane 0 of each warp: this warp's rows of round j.  Every round completes
+    // one phase of the warp's barrier (a plain arrive where nothing is
+    // copied), so its phases stay in step with the rounds.
     auto issue_rows = [&](int j) {
         if constexpr (kTMA) {
             if (j >= p.rounds) return;
-            const int buf = j % NB;
-            uint64_t* bar = mbar + buf * NW + warp;
+            uint64_t* bar = mbar + warp;
             if (chunk_len(j, warp) > 0) {
                 const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
                 mbar_arrive_expect_tx(bar, 2u * kChunkBytes);
-                tma_load_3d(rows_k(buf), &tmk, (int)c0, t, b, bar);
-                tma_load_3d(rows_v(buf), &tmv, (int)c0, t, b, bar);
+                tma_load_3d(kr, &tmk, (int)c0, t, b, bar);
+                tma_load_3d(vr, &tmv, (int)c0, t, b, bar);
             } else {
                 mbar_arrive(bar);
             }
@@ -244,10 +244,9 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     const uint32_t agg_bytes = (uint32_t)NC * 32u * 32u;
     if (warp == 0) tmem_alloc(tslot, (uint32_t)lay.tmem_cols());
     if (threadIdx.x == 0) {
-        mbar_init(abar, 1);
-        mbar_init(abar + 1, 1);
+        for (int r = 0; r < kAS; ++r) mbar_init(abar + r, 1);
         fence_mbar_init();
-        for (int r = 0; r < 2 && r < p.rounds; ++r) mbar_arrive_expect_tx(abar + r, agg_bytes);
+        for (int r = 0; r < kAS && r < p.rounds; ++r) mbar_arrive_expect_tx(abar + r, agg_bytes);
     }
     if constexpr (kTMA) {
         if (lane == 0) {
@@ -257,7 +256,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                 prefetch_tmap(&tmv);
                 prefetch_tmap(&tmy);
             }
-            for (int buf = 0; buf < NB; ++buf) mbar_init(mbar + buf * NW + warp, 1);
+            mbar_init(mbar + warp, 1);
             fence_mbar_init();
             if (warp == 0 && bulk) {
                 const uint32_t nb = Cg * 4;
@@ -271,7 +270,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                     bulk_load(sw + 4 * Cg, p.state_in + 2 * p.BC + ch, nb, pbar);
                 }
             }
-            for (int j = 0; j < NB; ++j) issue_rows(j);
+            issue_rows(0);
         }
         __syncwarp();
     }
@@ -295,8 +294,11 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     // just before it)
     cluster_arrive_relaxed();
     const uint32_t tbase = *tslot;
-    // this warp's stash: its lane quarter, 4 L columns for each warp of the quarter
-    const uint32_t taddr = tbase + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((warp >> 2) * 4 * L);
+    // this warp's stash in slot s: its lane quarter, NW L columns a slot,
+    // 4 L for each warp of the quarter
+    auto taddr = [&](int s) -> uint32_t {
+        return tbase + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(s * NW * L + (warp >> 2) * 4 * L);
+    };
     bool failed = false;
     if (bulk) {
         if (!mbar_wait_bounded(pbar, 0)) {
@@ -314,15 +316,15 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     }
     pair_derive(cc);
 
-    for (int round = 0; round < p.rounds; ++round) {
-        const int buf = round % NB;
+    // ---- 1. summary pass of a round: this warp's chunk summary into its
+    //         entry of summary slot round & 1 (kMulti) and its stash into
+    //         tensor-memory slot round & 1; then its rows take the next round's
+    auto summary = [&](int round) -> PairRef {
+        const int slot = kMulti ? (round & 1) : 0;
         const int n = chunk_len(round, warp);
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;  // segment start
-        IO* kr = rows_k(buf);
-        IO* vr = rows_v(buf);
         if constexpr (kTMA) {
-            if (n > 0 && !failed &&
-                !mbar_wait_bounded(mbar + buf * NW + warp, (uint32_t)((round / NB) & 1))) {
+            if (n > 0 && !failed && !mbar_wait_bounded(mbar + warp, (uint32_t)(round & 1))) {
                 failed = true;
                 if (lane == 0) atomicOr(&g_device_error, kErrTmaWait);
             }
@@ -342,56 +344,67 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
             }
             __syncwarp();
         }
-
-        // ---- 1. chunk summary and stash; then the rows are free
         PairRef ref;
         St sum[2];
-        chunk_phase1<IO, L, true>(ref, kr, vr, Cg, col, n, cc, sum, taddr);
+        chunk_phase1<IO, L, true>(ref, kr, vr, Cg, col, n, cc, sum, taddr(slot));
+        const TripleRef sums = triples(base + lay.sums(slot), NW * Cg);
 #pragma unroll
         for (int j = 0; j < 2; ++j) sums.put(warp * Cg + col + j, sum[j]);
-        if constexpr (kTMA && Lay::kOwnY) {
-            __syncwarp();  // every lane has read the rows: they take round + NB's
-            if (lane == 0) issue_rows(round + NB);
+        if constexpr (kTMA && kMulti) {
+            __syncwarp();  // every lane has read the rows
+            if (lane == 0) issue_rows(round + 1);
         }
-        __syncthreads();
+        return ref;
+    };
 
-        // ---- 2. warp 0: exclusive prefix of the chunk summaries (in place); the
-        //         segment aggregate goes by asynchronous DSMEM stores into slot
-        //         [round & 1][rank] of every CTA of the cluster, each store
-        //         completing bytes on that CTA's barrier of the slot
-        const int slot = round & 1;
-        const TripleRef agg = triples(base + lay.agg(slot), NC * Cg);
+    // ---- 2. warp 0, once every warp's summary of the round is in: exclusive
+    //         prefix of the chunk summaries (in place); the segment aggregate
+    //         goes by asynchronous DSMEM stores into slot [round % kAS][rank] of
+    //         every CTA of the cluster, each store completing bytes on that
+    //         CTA's barrier of the slot
+    auto scan_push = [&](int round) {
+        const int slot = kMulti ? (round & 1) : 0;
+        const TripleRef sums = triples(base + lay.sums(slot), NW * Cg);
+        const TripleRef agg = triples(base + lay.agg(round % kAS), NC * Cg);
+        const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
         // steps of this CTA's segment (the chunks' lengths follow from it)
         const int rem = (int)max((int64_t)0, min((int64_t)Ts, T - t0));
-        if (round == 0) cluster_wait();  // every CTA of the cluster has started
-        if (warp == 0) {
-            St acc[2];
-            if (NW == 8) {
-                scan_chunks<8, L>(sums, col, rem, cc, acc);
-            } else {
-                scan_chunks<4, L>(sums, col, rem, cc, acc);
-            }
-            const int off = rank * Cg + col;
-            const uint32_t la = smem_u32(agg.a + off), lb = smem_u32(agg.b + off);
-            const uint32_t lp = smem_u32(agg.p + off), lbar = smem_u32(abar + slot);
-#pragma unroll 1
-            for (int q = 0; q < NC; ++q) {
-                const uint32_t rbar = mapa_u32(lbar, (uint32_t)q);
-                st_async_v2f32(mapa_u32(la, (uint32_t)q), acc[0].a, acc[1].a, rbar);
-                st_async_v2f32(mapa_u32(lb, (uint32_t)q), acc[0].b, acc[1].b, rbar);
-                st_async_v2f64(mapa_u32(lp, (uint32_t)q), acc[0].p, acc[1].p, rbar);
-            }
+        St acc[2];
+        if (NW == 8) {
+            scan_chunks<8, L>(sums, col, rem, cc, acc);
+        } else {
+            scan_chunks<4, L>(sums, col, rem, cc, acc);
         }
-        __syncthreads();  // the exclusive prefixes are in place
+        const int off = rank * Cg + col;
+        const uint32_t la = smem_u32(agg.a + off), lb = smem_u32(agg.b + off);
+        const uint32_t lp = smem_u32(agg.p + off), lbar = smem_u32(abar + round % kAS);
+#pragma unroll 1
+        for (int q = 0; q < NC; ++q) {
+            const uint32_t rbar = mapa_u32(lbar, (uint32_t)q);
+            st_async_v2f32(mapa_u32(la, (uint32_t)q), acc[0].a, acc[1].a, rbar);
+            st_async_v2f32(mapa_u32(lb, (uint32_t)q), acc[0].b, acc[1].b, rbar);
+            st_async_v2f64(mapa_u32(lp, (uint32_t)q), acc[0].p, acc[1].p, rbar);
+        }
+    };
 
-        // ---- 3. every warp folds the round's aggregates once they have landed
-        if (!failed && !mbar_wait_cluster_bounded(abar + slot, (uint32_t)((round >> 1) & 1))) {
+    // ---- 3 and 4, once the round's prefixes are in place: every warp folds
+    //         the round's aggregates once they have landed, then emits its
+    //         chunk's outputs from the stash
+    auto finish = [&](int round, const PairRef& ref) {
+        const int slot = kMulti ? (round & 1) : 0, as = round % kAS;
+        const int n = chunk_len(round, warp);
+        const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
+        const TripleRef agg = triples(base + lay.agg(as), NC * Cg);
+        if (!failed && !mbar_wait_cluster_bounded(abar + as, (uint32_t)((round / kAS) & 1))) {
             failed = true;
             if (lane == 0) atomicOr(&g_device_error, kErrExchangeWait);
         }
-        // the slot's next use is round + 2: its pushes follow this CTA's own
-        // push of round + 1, so the barrier is re-armed well before them
-        if (threadIdx.x == 0 && round + 2 < p.rounds) mbar_arrive_expect_tx(abar + slot, agg_bytes);
+        // The slot's next use is round + 3.  Every CTA pushes round + 3 only
+        // after its fold of round + 2, so after this CTA's push of round + 2,
+        // which warp 0 issues after its CTA barrier of round + 1, which every
+        // warp reaches after this fold: the slot is read before it is
+        // overwritten, and re-armed (here) before it is written.
+        if (threadIdx.x == 0 && round + kAS < p.rounds) mbar_arrive_expect_tx(abar + as, agg_bytes);
         St P[2];
         {
             const int64_t rrem = T - (t0 - (int64_t)rank * Ts);  // steps of the round from segment 0 on
@@ -402,8 +415,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                 default: fold_aggs<8>(agg, col, rank, rrem, Ts, cc, carry, P); break;
             }
         }
-
-        // ---- 4. outputs of this warp's chunk
+        const TripleRef sums = triples(base + lay.sums(slot), NW * Cg);
         St S[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
@@ -411,18 +423,13 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         const int64_t cpair = c0 + col;
         const int64_t row0 = ((int64_t)b * T + t0 + warp * L) * C + cpair;  // k, v, y offset
         const bool ok0 = cpair < C, ok1 = cpair + 1 < C;
-        if constexpr (kTMA) {
-            // y staged (in place of k, or in the staging tile once the previous
-            // round's store has read it), sent out by one TMA store
-            IO* yr = Lay::kOwnY ? ystage : kr;
-            if (Lay::kOwnY && round > 0) {
-                if (lane == 0) bulk_wait_read_all();
-                __syncwarp();
-            }
+        if constexpr (kTMA && !kMulti) {
+            // one round: y staged in place of k, sent out by one TMA store
+            IO* yr = kr;
             auto st_one = [=](int s, int j, float y) { yr[s * Cg + col + j] = Io<IO>::from_f(y); };
             auto st_pair = [=](int s, f2 y) { Pair<IO>::store(yr + s * Cg + col, y); };
-            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr, kg + row0, vg + row0, C, ok0, ok1, st_pair,
-                                      st_one);
+            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
+                                      st_pair, st_one);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -432,6 +439,19 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                 }
             }
             __syncwarp();
+        } else if constexpr (kTMA) {
+            // several rounds (the rows already hold the next round's): y
+            // straight from registers, one 2-channel store a step per lane
+            // (C % 4 == 0 with TMA, so a pair in range is whole and aligned)
+            IO* yrow = yg + row0;
+            auto out_one = [=](int s, int j, float y) {
+                if (j == 0 ? ok0 : ok1) yrow[(int64_t)s * C + j] = Io<IO>::from_f(y);
+            };
+            auto out_pair = [=](int s, f2 y) {
+                if (ok0) Pair<IO>::store(yrow + (int64_t)s * C, y);
+            };
+            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
+                                      out_pair, out_one);
         } else {
             // element-wise stores (any alignment)
             IO* yrow = yg + row0;
@@ -442,11 +462,34 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
                 if (ok0) yrow[(int64_t)s * C] = Io<IO>::from_f(lo(y));
                 if (ok1) yrow[(int64_t)s * C + 1] = Io<IO>::from_f(hi(y));
             };
-            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr, kg + row0, vg + row0, C, ok0, ok1, out_pair,
-                                      out_one);
+            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
+                                      out_pair, out_one);
+        }
+    };
+
+    PairRef ref_cur = summary(0);
+    __syncthreads();  // every summary of round 0 is in
+    cluster_wait();   // every CTA of the cluster has started
+    if (warp == 0) scan_push(0);
+    if constexpr (!kMulti) {
+        // one round (the launch guarantees it)
+        __syncthreads();  // the exclusive prefixes are in place
+        finish(0, ref_cur);
+    } else {
+        // round + 1's summary pass while round's aggregates are on their way;
+        // one CTA barrier a round: after it round's prefixes (warp 0's scan,
+        // issued in the previous round) and round + 1's summaries are in
+        for (int round = 0; round < p.rounds; ++round) {
+            const bool more = round + 1 < p.rounds;
+            PairRef ref_next = ref_cur;
+            if (more) ref_next = summary(round + 1);
+            __syncthreads();
+            finish(round, ref_cur);
+            if (more && warp == 0) scan_push(round + 1);
+            ref_cur = ref_next;
         }
     }
-    if (kTMA && lane == 0) bulk_wait_read_all();  // staged rows stay valid until read
+    if (kTMA && !kMulti && lane == 0) bulk_wait_read_all();  // staged rows stay valid until read
 
     if (rank == 0 && warp == 0 && p.state_out) {
 #pragma unroll

@@ -101,6 +101,26 @@ def test_extreme_decay_and_bonus(cuda_device, variant):
     check(x, "f32", y, s, f"extreme/{VNAMES[variant]}")
 
 
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("variant", VARIANTS, ids=lambda v: VNAMES[v])
+def test_lifted_state_with_fast_decay(cuda_device, variant, dt):
+    """A carried state 43.5 nats above a chunk whose k spans 54.5 nats, under
+    decays of 5 to 9 nats a step: the state's weight after i steps,
+    e^{43.5 - i |w|}, is still comparable with the chunk's own denominator
+    (about e^{-54.5}) where e^{i w} alone is below the smallest float."""
+    B, T, C = 1, 96, 64
+    x = synth.custom(B, T, C, dt, seed=11, random_state=True)
+    x["w"][:] = -torch.linspace(5.0, 9.0, C, dtype=torch.float32)
+    x["u"][:] = 0.0
+    x["k"][:, :32, :] = -54.5
+    x["k"][:, 0, :] = 0.0
+    x["state_in"][2] = 43.5
+    x["state_in"][1] = 1.3
+    x["state_in"][0] = 0.9
+    y, s = gpu_forward(x, cuda_device, variant)
+    check(x, dt, y, s, f"lifted/{dt}/{VNAMES[variant]}")
+
+
 def test_misaligned_pointers_take_elementwise_path(cuda_device):
     B, T, C = 2, 300, 64
     x = synth.custom(B, T, C, "f16", seed=9, random_state=True)
