@@ -19,8 +19,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <climits>
 #include <atomic>
+#include <climits>
 #include <cstdlib>
 #include <cstring>
 
@@ -75,12 +75,6 @@ Geom seq_geom(int dtype) {
     return seq_geom_t<WKV4_SEQ_BF16>();
 }
 
-static int sm_count() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
-}
-
 static int env_int(const char* name, int dflt) {
     const char* e = std::getenv(name);
     return e ? std::atoi(e) : dflt;
@@ -114,41 +108,99 @@ template <> struct ScanL<float> { static constexpr int L = 16; };
 
 constexpr int kNwChoices[2] = {8, 4};  // warps per CTA, in order of preference
 
-// Resident CTAs per SM of one scan instantiation for each warp count, cached
-// per device (0: that warp count does not fit, or more CTAs would share an
-// SM than its tensor memory serves).
-struct ScanOcc {
-    std::atomic<int> bps[64][2];
+// Never launched: its occupancy under a given block size and shared-memory
+// request stands in for a scan kernel's cluster placement.
+__global__ void wkv4_occupancy_stand_in() {}
+
+// Clusters of nc CTAs of nthreads threads the GPU holds at once when every
+// SM holds at most bps of them (cached per device).
+struct ClusterFit {
+    std::atomic<int> n[64][2][4][4];  // [device][warp-count index][log2 nc][bps - 1]
 };
 
-template <typename IO, int L, bool kMulti, bool kTMA>
-static cudaError_t scan_occupancy(int (&bps)[2]) {
+static cudaError_t clusters_fit(int nwi, int nc, int bps, int& out) {
+    static ClusterFit fit;
     static DeviceFlags attr;
-    static ScanOcc occ;
+    out = 0;
+    if (bps <= 0) return cudaSuccess;
+    bps = bps > 4 ? 4 : bps;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const int lnc = nc == 1 ? 0 : nc == 2 ? 1 : nc == 4 ? 2 : 3;
+    std::atomic<int>& slot = fit.n[dev][nwi][lnc][bps - 1];
+    int v = slot.load(std::memory_order_acquire);
+    if (v == 0) {
+        if ((e = ensure_smem_attr(attr, wkv4_occupancy_stand_in, kMaxSmem)) != cudaSuccess) return e;
+        int per_sm = 233472, reserved = 1024;
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+        // the request at which bps, and not bps + 1, CTAs fit on an SM
+        size_t req = (size_t)per_sm / (size_t)(bps + 1) + 1;
+        req = req > (size_t)reserved ? req - (size_t)reserved : 0;
+        if (req > kMaxSmem) req = kMaxSmem;
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)nc, 1, 1);
+        cfg.blockDim = dim3((unsigned)(32 * kNwChoices[nwi]), 1, 1);
+        cfg.dynamicSmemBytes = req;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = (unsigned)nc;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if ((e = cudaOccupancyMaxActiveClusters(&n, wkv4_occupancy_stand_in, &cfg)) != cudaSuccess)
+            return e;
+        v = n > 0 ? n : -1;
+        slot.store(v, std::memory_order_release);
+    }
+    out = v > 0 ? v : 0;
+    return cudaSuccess;
+}
+
+// CTAs of one scan instantiation an SM holds, for nw warps and clusters of nc:
+// the least of its registers, shared memory (the request, which the tensor
+// memory cap may have raised), threads and tensor-memory columns.  Worked out
+// here rather than asked of the runtime, whose per-SM occupancy query
+// reports one CTA for these kernels where the SM holds two.
+template <typename IO, int L, bool kMulti, bool kTMA>
+static cudaError_t scan_ctas_per_sm(int nw, int nc, int& bps) {
+    static DeviceFlags attr;
+    static std::atomic<int> regs_cache[64];
+    bps = 0;
     auto kern = wkv4_scan_kernel<IO, L, kMulti, kTMA>;
     cudaError_t e = ensure_smem_attr(attr, kern, kMaxSmem);
     if (e != cudaSuccess) return e;
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    for (int i = 0; i < 2; ++i) {
-        int v = occ.bps[dev][i].load(std::memory_order_acquire);
-        if (v == 0) {
-            v = -1;
-            // the largest cluster's layout: a bound for every cluster size
-            const ScanLayout<IO, L, kMulti> lay{kNwChoices[i], kMaxCluster};
-            const size_t req = scan_smem_request(lay.bytes(), lay.tmem_cols());
-            if (req <= kMaxSmem) {
-                int n = 0;
-                if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * kNwChoices[i],
-                                                                       req)) != cudaSuccess)
-                    return e;
-                if (n > 0 && n * lay.tmem_cols() <= kTmemColumns) v = n;
-            }
-            occ.bps[dev][i].store(v, std::memory_order_release);
-        }
-        bps[i] = v > 0 ? v : 0;
+    int regs = regs_cache[dev].load(std::memory_order_acquire);
+    if (regs == 0) {
+        cudaFuncAttributes fa;
+        if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+        regs = fa.numRegs > 0 ? fa.numRegs : 1;
+        regs_cache[dev].store(regs, std::memory_order_release);
     }
+    const ScanLayout<IO, L, kMulti> lay{nw, nc};
+    const size_t req = scan_smem_request(lay.bytes(), lay.tmem_cols());
+    if (req > kMaxSmem || lay.tmem_cols() > kTmemColumns) return cudaSuccess;
+    int per_sm = 233472, reserved = 1024, reg_file = 65536, max_thr = 2048, max_blk = 32;
+    cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaDeviceGetAttribute(&reg_file, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&max_thr, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+    cudaDeviceGetAttribute(&max_blk, cudaDevAttrMaxBlocksPerMultiprocessor, dev);
+    const int warp_regs = ((regs * 32 + 255) / 256) * 256;  // allocated per warp in 256s
+    int n = reg_file / (warp_regs * nw);
+    n = std::min(n, (int)((size_t)per_sm / (req + (size_t)reserved)));
+    n = std::min(n, max_thr / (32 * nw));
+    n = std::min(n, kTmemColumns / lay.tmem_cols());
+    n = std::min(n, max_blk);
+    bps = n > 0 ? n : 0;
     return cudaSuccess;
 }
 
@@ -164,12 +216,8 @@ struct ScanShape {
 
 template <typename IO, int L, bool kTMA>
 static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
-    int b1[2], b2[2];  // one round, several rounds
-    cudaError_t e = scan_occupancy<IO, L, false, kTMA>(b1);
-    if (e != cudaSuccess) return e;
-    if ((e = scan_occupancy<IO, L, true, kTMA>(b2)) != cudaSuccess) return e;
-    const int sms = sm_count();
     const int force_nw = env_int("WKV4_SCAN_NW", 0), force_nc = env_int("WKV4_SCAN_CLUSTER", 0);
+    cudaError_t e = cudaSuccess;
     for (int i = 0; i < 2; ++i) {
         const int nw = kNwChoices[i];
         if (force_nw && nw != force_nw) continue;
@@ -180,12 +228,23 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
         } else if (nseg <= kMaxCluster) {
             while (nc < nseg) nc *= 2;
         } else {
-            const int64_t cap = (int64_t)b2[i] * sms;
-            while (nc < kMaxCluster && tiles * nc * 2 <= cap) nc *= 2;
+            for (int c = kMaxCluster; c > 1; c /= 2) {
+                int bps = 0, fit = 0;
+                if ((e = scan_ctas_per_sm<IO, L, true, kTMA>(nw, c, bps)) != cudaSuccess) return e;
+                if ((e = clusters_fit(i, c, bps, fit)) != cudaSuccess) return e;
+                if ((int64_t)fit >= tiles) {
+                    nc = c;
+                    break;
+                }
+            }
         }
         const int64_t rounds = (nseg + nc - 1) / nc;
         if (rounds > (1ll << 30)) continue;
-        if ((rounds == 1 ? b1[i] : b2[i]) <= 0) continue;  // does not fit on an SM
+        int bps = 0;
+        e = rounds == 1 ? scan_ctas_per_sm<IO, L, false, kTMA>(nw, nc, bps)
+                        : scan_ctas_per_sm<IO, L, true, kTMA>(nw, nc, bps);
+        if (e != cudaSuccess) return e;
+        if (bps <= 0) continue;  // does not fit on an SM
         out = {nw, nc, (int)rounds};
         return cudaSuccess;
     }
