@@ -11,23 +11,27 @@
 //   1. every warp summarises its chunk from the empty state (chunk_phase1
 //      with stash: the per-step numerators and denominators of its outputs
 //      go to tensor memory);
-//   2. warp 0 scans the NW chunk summaries (the state contribution before
-//      each chunk, the segment's aggregate) and pushes the aggregate into the
-//      shared memory of every CTA of the cluster by asynchronous DSMEM stores
-//      that complete on the receiving CTA's barrier of that round's slot;
-//   3. once all NC aggregates of the round have landed, every warp folds
-//      them, from the state carried into the round, into the state at the
-//      segment start and the state carried into the next round;
-//   4. every warp computes its chunk's outputs from the stash.
+//   2. once every summary is in, warp 0 scans them (the state contribution
+//      before each chunk, in place, and the segment's aggregate) and pushes
+//      the aggregate into the shared memory of every CTA of the cluster by
+//      asynchronous DSMEM stores that complete on the receiving CTA's
+//      barrier of that round's slot;
+//   3. once all NC aggregates of the round have landed, warp 1 folds them,
+//      from the state carried into the round, into the state at the segment
+//      start (into shared memory) and the state carried into the next round;
+//   4. after a CTA barrier every warp joins the segment start state with its
+//      chunk's prefix and computes its chunk's outputs from the stash.
+// Only warps 0 and 1 run the scan and the fold: every warp running them
+// would queue on the transcendental and conversion pipe they lean on.
 // One round: y is staged in the warp's k rows and sent out by one TMA store.
 // Several rounds (kMulti) are software-pipelined: a warp's rows take the next
-// round's load right after its summary pass; round r + 1's summary pass runs
-// before round r's steps 3 and 4, and warp 0 scans and pushes round r + 1
-// right after its step 4 of round r, so the aggregates travel while the
-// other warps work.  The chunk summaries and the stash alternate between two
-// slots, the aggregates rotate through three; y goes straight from registers
-// to global memory.  There is no global scratch: all exchange is through
-// cluster shared memory.  Every wait is bounded.
+// round's load right after its summary pass; round r + 1's steps 1 and 2 run
+// before round r's step 4, and warp 1 folds round r + 1 after its step 4 of
+// round r, so the aggregates travel while the warps work.  The chunk
+// summaries, the stash, the segment start state and the aggregates alternate
+// between two slots; y goes straight from registers to global memory.  There
+// is no global scratch: all exchange is through cluster shared memory.  Every
+// wait is bounded.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -47,16 +51,16 @@ constexpr int kMaxCluster = 8;  // cluster sizes 1, 2, 4, 8; warps per CTA 4 or 
 
 // Shared-memory layout for nw warps and clusters of nc (offsets from a
 // 128-byte aligned base): one buffer of k and v rows, the chunk summaries,
-// the tile's w, u and state, barriers, the aggregate slots.  kMulti (T walked
-// in several rounds, software-pipelined): two slots of chunk summaries and of
-// the stash, three of aggregates.
+// the state at the segment start, the aggregate slots, the tile's w, u and
+// state, barriers.  kMulti (T walked in several rounds, software-pipelined):
+// two slots of each of the chunk summaries, the stash, the segment start
+// state and the aggregates.
 template <typename IO, int L, bool kMulti>
 struct ScanLayout {
     static constexpr int kCg = 64;  // channels per tile: 32 lanes x 2
     static constexpr int kChunkBytes = L * kCg * (int)sizeof(IO);  // one warp's rows, one tensor
     static constexpr int kAlign = 128;                               // TMA destinations
-    static constexpr int kSlots = kMulti ? 2 : 1;                    // summaries, stash
-    static constexpr int kAggSlots = kMulti ? 3 : 1;
+    static constexpr int kSlots = kMulti ? 2 : 1;
     static_assert(L <= 256 && L % 4 == 0, "TMA box dims, stash column groups");
     static_assert(kChunkBytes % kAlign == 0, "TMA destination alignment");
     int nw, nc;
@@ -66,13 +70,16 @@ struct ScanLayout {
     __host__ __device__ size_t sums(int slot) const {  // [kSlots][nw][Cg] x 16 B
         return 2 * tile() + (size_t)slot * nw * kCg * 16;
     }
-    __host__ __device__ size_t params() const { return sums(kSlots); }  // [5][Cg] f32
-    __host__ __device__ size_t agg(int slot) const {                    // [kAggSlots][nc][Cg] x 16 B
-        return params() + (size_t)5 * kCg * 4 + (size_t)slot * nc * kCg * 16;
+    __host__ __device__ size_t start(int slot) const {  // [kSlots][Cg] x 16 B
+        return sums(kSlots) + (size_t)slot * kCg * 16;
     }
-    // rows [nw], params, aggregate slots [kAggSlots] x 8 B
-    __host__ __device__ size_t bars() const { return agg(kAggSlots); }
-    __host__ __device__ size_t tslot() const { return bars() + (size_t)(nw + 1 + kAggSlots) * 8; }
+    __host__ __device__ size_t agg(int slot) const {  // [kSlots][nc][Cg] x 16 B
+        return start(kSlots) + (size_t)slot * nc * kCg * 16;
+    }
+    __host__ __device__ size_t params() const { return agg(kSlots); }  // [5][Cg] f32
+    // rows [nw], params, aggregate slots [kSlots] x 8 B
+    __host__ __device__ size_t bars() const { return params() + (size_t)5 * kCg * 4; }
+    __host__ __device__ size_t tslot() const { return bars() + (size_t)(nw + 1 + kSlots) * 8; }
     __host__ __device__ size_t bytes() const { return kAlign + tslot() + 8; }
     // tensor-memory columns: 4 a step for each warp and slot, warps w and
     // w + 4 sharing a lane quarter
@@ -151,18 +158,17 @@ __device__ __forceinline__ void scan_chunks(const TripleRef& sums, int col, int 
     }
 }
 
-// Every warp: fold of the NC segment aggregates of a round into the state at
-// this CTA's segment start (P) and the state carried into the next round
-// (carry); segment q spans clamp(rrem - q Ts, 0, Ts) steps.
+// Warp 1: fold of the NC segment aggregates of a round into the state at this
+// CTA's segment start (P) and the state carried into the next round (carry);
+// segment q spans clamp(rrem - q Ts, 0, Ts) steps.
 template <int NC>
 __device__ __forceinline__ void fold_aggs(const TripleRef& agg, int col, int rank, int64_t rrem,
                                           int Ts, const PairConsts& cc, St (&carry)[2], St (&P)[2]) {
-    constexpr int Cg = 64;
     St y[NC][2];
 #pragma unroll
     for (int q = 0; q < NC; ++q)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) y[q][j] = agg.get(q * Cg + col + j);
+        for (int j = 0; j < 2; ++j) y[q][j] = agg.get(q * 64 + col + j);
     P[0] = carry[0];
     P[1] = carry[1];
 #pragma unroll
@@ -181,7 +187,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     wkv4_scan_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __grid_constant__ CUtensorMap tmy, const ScanParams p) {
     using Lay = ScanLayout<IO, L, kMulti>;
-    constexpr int kAS = Lay::kAggSlots;
+    constexpr int kAS = Lay::kSlots;  // aggregate slots
     constexpr int Cg = Lay::kCg;
     constexpr int kChunkBytes = Lay::kChunkBytes;
     constexpr unsigned kAlign = Lay::kAlign;
@@ -275,7 +281,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         __syncwarp();
     }
     PairConsts cc;
-    St carry[2];  // every warp: the state carried into the current round
+    St carry[2];  // the state carried into the current round (warp 1 folds it)
     if (!bulk) {
         pair_wu(p.w, p.u, c0 + col, C, cc);
 #pragma unroll
@@ -363,8 +369,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     //         every CTA of the cluster, each store completing bytes on that
     //         CTA's barrier of the slot
     auto scan_push = [&](int round) {
-        const int slot = kMulti ? (round & 1) : 0;
-        const TripleRef sums = triples(base + lay.sums(slot), NW * Cg);
+        const TripleRef sums = triples(base + lay.sums(kMulti ? (round & 1) : 0), NW * Cg);
         const TripleRef agg = triples(base + lay.agg(round % kAS), NC * Cg);
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
         // steps of this CTA's segment (the chunks' lengths follow from it)
@@ -387,39 +392,56 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         }
     };
 
-    // ---- 3 and 4, once the round's prefixes are in place: every warp folds
-    //         the round's aggregates once they have landed, then emits its
-    //         chunk's outputs from the stash
-    auto finish = [&](int round, const PairRef& ref) {
-        const int slot = kMulti ? (round & 1) : 0, as = round % kAS;
-        const int n = chunk_len(round, warp);
+    // ---- 3. warp 1, once the round's aggregates have landed: the state at
+    //         this CTA's segment start (the state carried into the round
+    //         joined with the aggregates of the segments before it) into
+    //         start slot round & 1, and the state carried into the next round
+    //         (joined with all of them).  Only warp 1 holds the carried state.
+    auto fold = [&](int round) {
+        const int as = round % kAS;
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
         const TripleRef agg = triples(base + lay.agg(as), NC * Cg);
         if (!failed && !mbar_wait_cluster_bounded(abar + as, (uint32_t)((round / kAS) & 1))) {
             failed = true;
             if (lane == 0) atomicOr(&g_device_error, kErrExchangeWait);
         }
-        // The slot's next use is round + 3.  Every CTA pushes round + 3 only
-        // after its fold of round + 2, so after this CTA's push of round + 2,
-        // which warp 0 issues after its CTA barrier of round + 1, which every
-        // warp reaches after this fold: the slot is read before it is
-        // overwritten, and re-armed (here) before it is written.
-        if (threadIdx.x == 0 && round + kAS < p.rounds) mbar_arrive_expect_tx(abar + as, agg_bytes);
+        // The slot's next use is round + 2.  Every CTA pushes round + 2 after
+        // its CTA barrier of round + 1, which follows its own fold of round
+        // + 1, which waited for this CTA's push of round + 1, issued after
+        // this CTA's barrier of round, which this warp reaches after this
+        // fold: the slot is read before it is overwritten, and re-armed (here)
+        // before it is written.
+        if (lane == 0 && round + kAS < p.rounds) mbar_arrive_expect_tx(abar + as, agg_bytes);
+        const int64_t rrem = T - (t0 - (int64_t)rank * Ts);  // steps of the round from segment 0 on
         St P[2];
-        {
-            const int64_t rrem = T - (t0 - (int64_t)rank * Ts);  // steps of the round from segment 0 on
-            switch (NC) {
-                case 1: fold_aggs<1>(agg, col, rank, rrem, Ts, cc, carry, P); break;
-                case 2: fold_aggs<2>(agg, col, rank, rrem, Ts, cc, carry, P); break;
-                case 4: fold_aggs<4>(agg, col, rank, rrem, Ts, cc, carry, P); break;
-                default: fold_aggs<8>(agg, col, rank, rrem, Ts, cc, carry, P); break;
-            }
+        switch (NC) {
+            case 1: fold_aggs<1>(agg, col, rank, rrem, Ts, cc, carry, P); break;
+            case 2: fold_aggs<2>(agg, col, rank, rrem, Ts, cc, carry, P); break;
+            case 4: fold_aggs<4>(agg, col, rank, rrem, Ts, cc, carry, P); break;
+            default: fold_aggs<8>(agg, col, rank, rrem, Ts, cc, carry, P); break;
         }
+        const TripleRef st = triples(base + lay.start(kMulti ? (round & 1) : 0), Cg);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) st.put(col + j, P[j]);
+    };
+
+    // ---- every warp, once the segment start state and the chunk prefixes of
+    //      the round are in place: the state at its chunk start
+    auto chunk_start = [&](int round, St (&S)[2]) {
+        const int slot = kMulti ? (round & 1) : 0;
+        const TripleRef st = triples(base + lay.start(slot), Cg);
         const TripleRef sums = triples(base + lay.sums(slot), NW * Cg);
-        St S[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-            S[j] = combine(P[j], sums.get(warp * Cg + col + j), (double)(warp * L) * cc.w2[j]);
+            S[j] = combine(st.get(col + j), sums.get(warp * Cg + col + j), (double)(warp * L) * cc.w2[j]);
+    };
+
+    // ---- 4. every warp: its chunk's outputs from the stash and the state S
+    //         at its start
+    auto emit = [&](int round, const PairRef& ref, const St (&S)[2]) {
+        const int slot = kMulti ? (round & 1) : 0;
+        const int n = chunk_len(round, warp);
+        const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
         const int64_t cpair = c0 + col;
         const int64_t row0 = ((int64_t)b * T + t0 + warp * L) * C + cpair;  // k, v, y offset
         const bool ok0 = cpair < C, ok1 = cpair + 1 < C;
@@ -473,25 +495,35 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     if (warp == 0) scan_push(0);
     if constexpr (!kMulti) {
         // one round (the launch guarantees it)
-        __syncthreads();  // the exclusive prefixes are in place
-        finish(0, ref_cur);
+        if (warp == 1) fold(0);
+        __syncthreads();  // the segment start state and the chunk prefixes are in place
+        St S[2];
+        chunk_start(0, S);
+        emit(0, ref_cur, S);
     } else {
-        // round + 1's summary pass while round's aggregates are on their way;
-        // one CTA barrier a round: after it round's prefixes (warp 0's scan,
-        // issued in the previous round) and round + 1's summaries are in
+        // Round r + 1's summary pass runs while round r's aggregates are on
+        // their way.  One CTA barrier a round (B_r): before it every warp has
+        // summarised its chunk of round r + 1, warp 0 has scanned and pushed
+        // round r, and warp 1 has folded round r; after it warp 0 scans and
+        // pushes round r + 1, every warp emits round r, and warp 1 folds round
+        // r + 1, whose aggregates have had a whole output pass to arrive.
         for (int round = 0; round < p.rounds; ++round) {
             const bool more = round + 1 < p.rounds;
             PairRef ref_next = ref_cur;
             if (more) ref_next = summary(round + 1);
+            if (round == 0 && warp == 1) fold(0);
             __syncthreads();
-            finish(round, ref_cur);
             if (more && warp == 0) scan_push(round + 1);
+            St S[2];
+            chunk_start(round, S);
+            emit(round, ref_cur, S);
+            if (more && warp == 1) fold(round + 1);
             ref_cur = ref_next;
         }
     }
     if (kTMA && !kMulti && lane == 0) bulk_wait_read_all();  // staged rows stay valid until read
 
-    if (rank == 0 && warp == 0 && p.state_out) {
+    if (rank == 0 && warp == 1 && p.state_out) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int64_t c = c0 + col + j;
