@@ -11,11 +11,13 @@
 //   1. every warp summarises its chunk from the empty state (chunk_phase1
 //      with stash: the per-step numerators and denominators of its outputs
 //      go to tensor memory);
-//   2. once every summary is in, warp 0 scans them (the state contribution
-//      before each chunk, in place, and the segment's aggregate) and pushes
-//      the aggregate into the shared memory of every CTA of the cluster by
-//      asynchronous DSMEM stores that complete on the receiving CTA's
-//      barrier of that round's slot;
+//   2. once every summary is in, warp 0 joins them (a balanced tree) into the
+//      segment's aggregate and pushes it into the shared memory of every CTA
+//      of the cluster by asynchronous DSMEM stores that complete on the
+//      receiving CTA's barrier of that round's slot; the state contribution
+//      before each chunk: one round, every warp joins the summaries before
+//      its own; several rounds, warp 0 scans them in place (one chain, which
+//      also gives the aggregate);
 //   3. once all NC aggregates of the round have landed, warp 1 folds them,
 //      from the state carried into the round, into the state at the segment
 //      start (into shared memory) and the state carried into the next round;
@@ -133,6 +135,69 @@ __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Stretches q = 0, 1, ... of a round held in shared memory as entries
+// q * 64 + col + j of t (the lane's channel pair j = 0, 1), stretch q spanning
+// len(q) steps (an empty stretch is the empty state), joined as a balanced
+// tree: depth log2 of their count instead of a left-to-right chain (the
+// combine is associative, so the result is the same up to rounding).
+
+// Stretches lo .. lo + S - 1 joined (lo warp-uniform): r, spanning n steps.
+template <int S, typename Len>
+__device__ __forceinline__ void tree_range(const TripleRef& t, int col, int lo, Len len,
+                                           const PairConsts& cc, St (&r)[2], int& n) {
+    if constexpr (S == 1) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) r[j] = t.get(lo * 64 + col + j);
+        n = len(lo);
+    } else {
+        St x[2], y[2];
+        int nx, ny;
+        tree_range<S / 2>(t, col, lo, len, cc, x, nx);
+        tree_range<S / 2>(t, col, lo + S / 2, len, cc, y, ny);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) r[j] = combine(x[j], y[j], (double)ny * cc.w2[j]);
+        n = nx + ny;
+    }
+}
+
+// Stretches 0 .. m - 1 of N joined (m warp-uniform, 0 <= m < N): the state
+// contribution before stretch m (the empty state for m = 0), spanning npre.
+template <int N, typename Len>
+__device__ __forceinline__ void tree_prefix(const TripleRef& t, int col, int m, Len len,
+                                            const PairConsts& cc, St (&pre)[2], int& npre) {
+    pre[0] = pre[1] = empty_state();
+    npre = 0;
+    int lo = 0;
+    auto add = [&](const St (&y)[2], int ny) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) pre[j] = combine(pre[j], y[j], (double)ny * cc.w2[j]);
+        npre += ny;
+    };
+    if constexpr (N >= 8) {
+        if (m & 4) {
+            tree_range<4>(t, col, 0, len, cc, pre, npre);
+            lo = 4;
+        }
+    }
+    if constexpr (N >= 4) {
+        if (m & 2) {
+            St y[2];
+            int ny;
+            tree_range<2>(t, col, lo, len, cc, y, ny);
+            add(y, ny);
+            lo += 2;
+        }
+    }
+    if constexpr (N >= 2) {
+        if (m & 1) {
+            St y[2];
+            int ny;
+            tree_range<1>(t, col, lo, len, cc, y, ny);
+            add(y, ny);
+        }
+    }
+}
+
 // Warp 0: exclusive prefix of the NW chunk summaries of a segment (in
 // place: entry q becomes the state before chunk q) and the segment aggregate
 // in acc.  All summaries are read before the chain starts; chunk q spans
@@ -248,7 +313,6 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     const bool bulk = kTMA && p.bulk_params && c0 + Cg <= C;
     // every CTA of the cluster pushes 32 B per lane into each aggregate slot
     const uint32_t agg_bytes = (uint32_t)NC * 32u * 32u;
-    if (warp == 0) tmem_alloc(tslot, (uint32_t)lay.tmem_cols());
     if (threadIdx.x == 0) {
         for (int r = 0; r < kAS; ++r) mbar_init(abar + r, 1);
         fence_mbar_init();
@@ -280,6 +344,8 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         }
         __syncwarp();
     }
+    // tensor memory after the loads are on their way
+    if (warp == 0) tmem_alloc(tslot, (uint32_t)lay.tmem_cols());
     PairConsts cc;
     St carry[2];  // the state carried into the current round (warp 1 folds it)
     if (!bulk) {
@@ -363,11 +429,12 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         return ref;
     };
 
-    // ---- 2. warp 0, once every warp's summary of the round is in: exclusive
-    //         prefix of the chunk summaries (in place); the segment aggregate
-    //         goes by asynchronous DSMEM stores into slot [round % kAS][rank] of
-    //         every CTA of the cluster, each store completing bytes on that
-    //         CTA's barrier of the slot
+    // ---- 2. warp 0, once every warp's summary of the round is in: the
+    //         segment aggregate (one round: the chunk summaries joined as a
+    //         tree; several rounds: with their exclusive prefix, in place, by
+    //         one chain) goes by asynchronous DSMEM stores into slot
+    //         [round % kAS][rank] of every CTA of the cluster, each store
+    //         completing bytes on that CTA's barrier of the slot
     auto scan_push = [&](int round) {
         const TripleRef sums = triples(base + lay.sums(kMulti ? (round & 1) : 0), NW * Cg);
         const TripleRef agg = triples(base + lay.agg(round % kAS), NC * Cg);
@@ -375,10 +442,20 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         // steps of this CTA's segment (the chunks' lengths follow from it)
         const int rem = (int)max((int64_t)0, min((int64_t)Ts, T - t0));
         St acc[2];
-        if (NW == 8) {
-            scan_chunks<8, L>(sums, col, rem, cc, acc);
+        if constexpr (kMulti) {
+            if (NW == 8) {
+                scan_chunks<8, L>(sums, col, rem, cc, acc);
+            } else {
+                scan_chunks<4, L>(sums, col, rem, cc, acc);
+            }
         } else {
-            scan_chunks<4, L>(sums, col, rem, cc, acc);
+            auto clen = [=](int q) { return max(0, min(L, rem - q * L)); };
+            int nacc;
+            if (NW == 8) {
+                tree_range<8>(sums, col, 0, clen, cc, acc, nacc);
+            } else {
+                tree_range<4>(sums, col, 0, clen, cc, acc, nacc);
+            }
         }
         const int off = rank * Cg + col;
         const uint32_t la = smem_u32(agg.a + off), lb = smem_u32(agg.b + off);
@@ -425,8 +502,9 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         for (int j = 0; j < 2; ++j) st.put(col + j, P[j]);
     };
 
-    // ---- every warp, once the segment start state and the chunk prefixes of
-    //      the round are in place: the state at its chunk start
+    // ---- several rounds, every warp, once the segment start state and the
+    //      chunk prefixes of the round are in place: the state at its chunk
+    //      start
     auto chunk_start = [&](int round, St (&S)[2]) {
         const int slot = kMulti ? (round & 1) : 0;
         const TripleRef st = triples(base + lay.start(slot), Cg);
@@ -434,6 +512,19 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
 #pragma unroll
         for (int j = 0; j < 2; ++j)
             S[j] = combine(st.get(col + j), sums.get(warp * Cg + col + j), (double)(warp * L) * cc.w2[j]);
+    };
+
+    // ---- one round, every warp, once every summary is in: the summaries of
+    //      the chunks before its own joined (E, spanning nE steps)
+    auto chunk_prefix = [&](St (&E)[2], int& nE) {
+        const TripleRef sums = triples(base + lay.sums(0), NW * Cg);
+        const int rem = (int)max((int64_t)0, min((int64_t)Ts, T - (int64_t)rank * Ts));
+        auto clen = [=](int q) { return max(0, min(L, rem - q * L)); };
+        if (NW == 8) {
+            tree_prefix<8>(sums, col, warp, clen, cc, E, nE);
+        } else {
+            tree_prefix<4>(sums, col, warp, clen, cc, E, nE);
+        }
     };
 
     // ---- 4. every warp: its chunk's outputs from the stash and the state S
@@ -494,11 +585,17 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     cluster_wait();   // every CTA of the cluster has started
     if (warp == 0) scan_push(0);
     if constexpr (!kMulti) {
-        // one round (the launch guarantees it)
+        // one round (the launch guarantees it); each warp joins the summaries
+        // before its chunk while the aggregates travel
+        St E[2];
+        int nE;
+        chunk_prefix(E, nE);
         if (warp == 1) fold(0);
-        __syncthreads();  // the segment start state and the chunk prefixes are in place
+        __syncthreads();  // the segment start state is in place
+        const TripleRef st = triples(base + lay.start(0), Cg);
         St S[2];
-        chunk_start(0, S);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) S[j] = combine(st.get(col + j), E[j], (double)nE * cc.w2[j]);
         emit(0, ref_cur, S);
     } else {
         // Round r + 1's summary pass runs while round r's aggregates are on
