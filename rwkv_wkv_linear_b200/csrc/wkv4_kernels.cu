@@ -204,14 +204,18 @@ static cudaError_t scan_ctas_per_sm(int nw, int nc, int& bps) {
     return cudaSuccess;
 }
 
-// Launch shape of the scan: warps per CTA (NW) and cluster size (NC).  8 warps
-// per CTA wherever it fits.  When T fits in at most 8 segments, one round
-// with NC = segments (rounded up to a power of two), even if the grid takes
-// several waves; when T needs several rounds, NC is the largest power of two
-// whose grid still fits in one wave (a second wave of CTAs that each walk all
-// of T would be costly).  WKV4_SCAN_NW / WKV4_SCAN_CLUSTER override (tuning).
+// Launch shape of the scan: warps per CTA (NW), cluster size (NC) and the
+// number of clusters.  8 warps per CTA wherever it fits.  When T fits in at
+// most 8 segments, one round with NC = segments (rounded up to a power of
+// two), and as many clusters as the GPU holds at once (at most one per
+// channel tile), each walking its share of the tiles; when T needs several
+// rounds, NC is the largest power of two whose grid of one cluster per tile
+// still fits in one wave (a second wave of CTAs that each walk all of T would
+// be costly).  WKV4_SCAN_NW / WKV4_SCAN_CLUSTER override NW / NC, and
+// WKV4_SCAN_WAVES=1 gives one cluster per tile with one round (tuning).
 struct ScanShape {
     int nw, nc, rounds;
+    int64_t clusters;
 };
 
 template <typename IO, int L, bool kTMA>
@@ -245,7 +249,13 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
                         : scan_ctas_per_sm<IO, L, true, kTMA>(nw, nc, bps);
         if (e != cudaSuccess) return e;
         if (bps <= 0) continue;  // does not fit on an SM
-        out = {nw, nc, (int)rounds};
+        int64_t clusters = tiles;
+        if (rounds == 1 && !env_int("WKV4_SCAN_WAVES", 0)) {
+            int fit = 0;
+            if ((e = clusters_fit(i, nc, bps, fit)) != cudaSuccess) return e;
+            if (fit > 0 && fit < tiles) clusters = fit;
+        }
+        out = {nw, nc, (int)rounds, clusters};
         return cudaSuccess;
     }
     return cudaErrorInvalidConfiguration;
@@ -253,7 +263,7 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
 
 template <typename IO, int L, bool kMulti, bool kTMA>
 static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const ScanShape& sh,
-                                  int64_t tiles, EncodeFn encode) {
+                                  EncodeFn encode) {
     CUtensorMap tk, tv, ty;
     std::memset(&tk, 0, sizeof(tk));
     std::memset(&tv, 0, sizeof(tv));
@@ -268,7 +278,7 @@ static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const S
     const ScanLayout<IO, L, kMulti> lay{sh.nw, sh.nc};
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)(tiles * sh.nc), 1, 1);
+    cfg.gridDim = dim3((unsigned)(sh.clusters * sh.nc), 1, 1);
     cfg.blockDim = dim3(32 * sh.nw, 1, 1);
     cfg.dynamicSmemBytes = scan_smem_request(lay.bytes(), lay.tmem_cols());
     cfg.stream = a.stream;
@@ -300,13 +310,15 @@ static cudaError_t launch_scan_t(const FwdArgs& a, EncodeFn encode) {
     p.bulk_params = ((uintptr_t)a.w % 16 == 0) && ((uintptr_t)a.u % 16 == 0) &&
                     ((uintptr_t)a.state_in % 16 == 0) && (a.C % 4 == 0);
     const int64_t tiles = a.B * p.CGB;
+    if (tiles > (1ll << 30)) return cudaErrorInvalidConfiguration;
     ScanShape sh;
     cudaError_t e = pick_scan_shape<IO, L, kTMA>(tiles, a.T, sh);
     if (e != cudaSuccess) return e;
-    if (tiles * sh.nc > (int64_t)INT32_MAX) return cudaErrorInvalidConfiguration;
+    if (sh.clusters * sh.nc > (int64_t)INT32_MAX) return cudaErrorInvalidConfiguration;
+    p.tiles = (int)tiles;
     p.rounds = sh.rounds;
-    if (sh.rounds == 1) return launch_scan_nb<IO, L, false, kTMA>(a, p, sh, tiles, encode);
-    return launch_scan_nb<IO, L, true, kTMA>(a, p, sh, tiles, encode);
+    if (sh.rounds == 1) return launch_scan_nb<IO, L, false, kTMA>(a, p, sh, encode);
+    return launch_scan_nb<IO, L, true, kTMA>(a, p, sh, encode);
 }
 
 cudaError_t launch_scan(const FwdArgs& a, bool tma, EncodeFn encode) {

@@ -46,23 +46,30 @@ namespace cg = cooperative_groups;
 
 constexpr int kMaxCluster = 8;  // cluster sizes 1, 2, 4, 8; warps per CTA 4 or 8
 
-// Register cap of the scan kernel: two CTAs of 8 warps per SM.
-#ifndef WKV4_SCAN_MAXNREG
-#define WKV4_SCAN_MAXNREG 128
-#endif
+// Register cap of the scan kernel: two CTAs of 8 warps per SM, except where
+// an 8-warp CTA's tensor memory (nw L columns a stash slot, two slots with
+// several rounds) takes more than half of the SM's 512 columns, so one CTA
+// per SM is all there is and the cap would only cost spills.
+template <int L, bool kMulti>
+constexpr int scan_maxnreg() {
+    return (kMulti && 2 * 8 * L > 256) ? 255 : 128;
+}
 
 // Shared-memory layout for nw warps and clusters of nc (offsets from a
 // 128-byte aligned base): one buffer of k and v rows, the chunk summaries,
-// the state at the segment start, the aggregate slots, the tile's w, u and
+// the state at the segment start, two aggregate slots, the tile's w, u and
 // state, barriers.  kMulti (T walked in several rounds, software-pipelined):
-// two slots of each of the chunk summaries, the stash, the segment start
-// state and the aggregates.
+// two slots of the chunk summaries, the stash and the segment start state.
+// One round (a cluster walks several channel tiles): two slots of w, u and
+// state, so that the next tile's come in while this one's are in use.
 template <typename IO, int L, bool kMulti>
 struct ScanLayout {
     static constexpr int kCg = 64;  // channels per tile: 32 lanes x 2
     static constexpr int kChunkBytes = L * kCg * (int)sizeof(IO);  // one warp's rows, one tensor
     static constexpr int kAlign = 128;                               // TMA destinations
-    static constexpr int kSlots = kMulti ? 2 : 1;
+    static constexpr int kSlots = kMulti ? 2 : 1;       // summaries, stash, start state
+    static constexpr int kAggSlots = 2;
+    static constexpr int kParamSlots = kMulti ? 1 : 2;
     static_assert(L <= 256 && L % 4 == 0, "TMA box dims, stash column groups");
     static_assert(kChunkBytes % kAlign == 0, "TMA destination alignment");
     int nw, nc;
@@ -75,13 +82,17 @@ struct ScanLayout {
     __host__ __device__ size_t start(int slot) const {  // [kSlots][Cg] x 16 B
         return sums(kSlots) + (size_t)slot * kCg * 16;
     }
-    __host__ __device__ size_t agg(int slot) const {  // [kSlots][nc][Cg] x 16 B
+    __host__ __device__ size_t agg(int slot) const {  // [kAggSlots][nc][Cg] x 16 B
         return start(kSlots) + (size_t)slot * nc * kCg * 16;
     }
-    __host__ __device__ size_t params() const { return agg(kSlots); }  // [5][Cg] f32
-    // rows [nw], params, aggregate slots [kSlots] x 8 B
-    __host__ __device__ size_t bars() const { return params() + (size_t)5 * kCg * 4; }
-    __host__ __device__ size_t tslot() const { return bars() + (size_t)(nw + 1 + kSlots) * 8; }
+    __host__ __device__ size_t params(int slot) const {  // [kParamSlots][5][Cg] f32
+        return agg(kAggSlots) + (size_t)slot * 5 * kCg * 4;
+    }
+    // rows [nw], params [kParamSlots], aggregate slots [kAggSlots] x 8 B
+    __host__ __device__ size_t bars() const { return params(kParamSlots); }
+    __host__ __device__ size_t tslot() const {
+        return bars() + (size_t)(nw + kParamSlots + kAggSlots) * 8;
+    }
     __host__ __device__ size_t bytes() const { return kAlign + tslot() + 8; }
     // tensor-memory columns: 4 a step for each warp and slot, warps w and
     // w + 4 sharing a lane quarter
@@ -91,6 +102,7 @@ struct ScanLayout {
 struct ScanParams {
     int64_t T, C;
     int CGB;     // channel tiles per batch row
+    int tiles;   // B * CGB
     int rounds;  // ceil(segments / NC)
     const float* w;
     const float* u;
@@ -248,11 +260,11 @@ __device__ __forceinline__ void fold_aggs(const TripleRef& agg, int col, int ran
 }
 
 template <typename IO, int L, bool kMulti, bool kTMA>
-__global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
+__global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     wkv4_scan_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __grid_constant__ CUtensorMap tmy, const ScanParams p) {
     using Lay = ScanLayout<IO, L, kMulti>;
-    constexpr int kAS = Lay::kSlots;  // aggregate slots
+    constexpr int kAS = Lay::kAggSlots;
     constexpr int Cg = Lay::kCg;
     constexpr int kChunkBytes = Lay::kChunkBytes;
     constexpr unsigned kAlign = Lay::kAlign;
@@ -265,16 +277,16 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     // align by offsetting the shared array itself (a round trip through an
     // integer would lose the address space and turn every access generic)
     unsigned char* base = smem_raw + ((kAlign - (smem_u32(smem_raw) & (kAlign - 1))) & (kAlign - 1));
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // rows [NW], params
-    uint64_t* pbar = mbar + NW;
-    uint64_t* abar = pbar + 1;  // [kAS]: the aggregates of a round have landed
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // rows [NW]
+    uint64_t* pbar = mbar + NW;                                       // params [kParamSlots]
+    uint64_t* abar = pbar + Lay::kParamSlots;  // [kAS]: the aggregates of a round have landed
     uint32_t* tslot = reinterpret_cast<uint32_t*>(base + lay.tslot());
-    float* sw = reinterpret_cast<float*>(base + lay.params());  // [5][Cg]: w, u, a, b, p
 
     const int rank = (int)cluster.block_rank();
-    const int g = blockIdx.x / NC;
-    const int b = g / p.CGB;
-    const int64_t c0 = (int64_t)(g - b * p.CGB) * Cg;
+    const int G = (int)(gridDim.x / NC);  // clusters
+    int tile = (int)(blockIdx.x / NC);    // this cluster's channel tile (its first, with one round)
+    int b = tile / p.CGB;
+    int64_t c0 = (int64_t)(tile - b * p.CGB) * Cg;
     const int64_t T = p.T, C = p.C;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int col = lane * 2;
@@ -282,6 +294,8 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     const IO* kg = static_cast<const IO*>(p.k);
     const IO* vg = static_cast<const IO*>(p.v);
     IO* yg = static_cast<IO*>(p.y);
+    // aggregate exchanges this cluster makes: one a round, or one a tile
+    const int items = kMulti ? p.rounds : (p.tiles - tile + G - 1) / G;
 
     auto chunk_len = [&](int j, int q) -> int {  // steps of chunk q of this CTA in round j
         const int64_t tc = (int64_t)j * seg_stride + (int64_t)rank * Ts + (int64_t)q * L;
@@ -289,74 +303,76 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     };
     IO* const kr = reinterpret_cast<IO*>(base + lay.k()) + warp * L * Cg;  // this warp's rows
     IO* const vr = reinterpret_cast<IO*>(base + lay.v()) + warp * L * Cg;
-    // Lane 0 of each warp: this warp's rows of round j.  Every round completes
-    // one phase of the warp's barrier (a plain arrive where nothing is
-    // copied), so its phases stay in step with the rounds.
-    auto issue_rows = [&](int j) {
+    // Lane 0 of each warp: this warp's rows of round j of the tile at (bb,
+    // cc0), k and v (issue_k announces both on the warp's barrier, issue_v may
+    // follow later).  Every round completes one phase of the barrier (a plain
+    // arrive where nothing is copied), so its phases stay in step.
+    auto issue_k = [&](int j, int bb, int64_t cc0) {
         if constexpr (kTMA) {
-            if (j >= p.rounds) return;
             uint64_t* bar = mbar + warp;
             if (chunk_len(j, warp) > 0) {
                 const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
                 mbar_arrive_expect_tx(bar, 2u * kChunkBytes);
-                tma_load_3d(kr, &tmk, (int)c0, t, b, bar);
-                tma_load_3d(vr, &tmv, (int)c0, t, b, bar);
+                tma_load_3d(kr, &tmk, (int)cc0, t, bb, bar);
             } else {
                 mbar_arrive(bar);
             }
         }
     };
+    auto issue_v = [&](int j, int bb, int64_t cc0) {
+        if constexpr (kTMA) {
+            if (chunk_len(j, warp) > 0) {
+                const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
+                tma_load_3d(vr, &tmv, (int)cc0, t, bb, mbar + warp);
+            }
+        }
+    };
+    auto issue_rows = [&](int j, int bb, int64_t cc0) {
+        issue_k(j, bb, cc0);
+        issue_v(j, bb, cc0);
+    };
+    // Per-channel w, u and the state of a tile: a full 64-channel slice with
+    // aligned pointers comes by bulk copy (lane 0 of warp 0) into a parameter
+    // slot, on that slot's barrier.
+    auto bulk_ok = [&](int64_t cc0) { return kTMA && p.bulk_params && cc0 + Cg <= C; };
+    auto issue_params = [&](int slot, int bb, int64_t cc0) {
+        float* sw = reinterpret_cast<float*>(base + lay.params(slot));
+        const uint32_t nb = Cg * 4;
+        const int64_t ch = (int64_t)bb * C + cc0;
+        mbar_arrive_expect_tx(pbar + slot, (p.state_in ? 5u : 2u) * nb);
+        bulk_load(sw, p.w + cc0, nb, pbar + slot);
+        bulk_load(sw + Cg, p.u + cc0, nb, pbar + slot);
+        if (p.state_in) {
+            bulk_load(sw + 2 * Cg, p.state_in + ch, nb, pbar + slot);
+            bulk_load(sw + 3 * Cg, p.state_in + p.BC + ch, nb, pbar + slot);
+            bulk_load(sw + 4 * Cg, p.state_in + 2 * p.BC + ch, nb, pbar + slot);
+        }
+    };
 
-    // Per-channel w, u and the state for this tile: a full 64-channel slice
-    // with aligned pointers comes by bulk copy on its own mbarrier, issued
-    // before the rows, so it does not queue behind other CTAs' row traffic.
-    const bool bulk = kTMA && p.bulk_params && c0 + Cg <= C;
     // every CTA of the cluster pushes 32 B per lane into each aggregate slot
     const uint32_t agg_bytes = (uint32_t)NC * 32u * 32u;
     if (threadIdx.x == 0) {
         for (int r = 0; r < kAS; ++r) mbar_init(abar + r, 1);
         fence_mbar_init();
-        for (int r = 0; r < kAS && r < p.rounds; ++r) mbar_arrive_expect_tx(abar + r, agg_bytes);
+        for (int r = 0; r < kAS && r < items; ++r) mbar_arrive_expect_tx(abar + r, agg_bytes);
     }
     if constexpr (kTMA) {
         if (lane == 0) {
             if (warp == 0) {
-                mbar_init(pbar, 1);
+                for (int s = 0; s < Lay::kParamSlots; ++s) mbar_init(pbar + s, 1);
                 prefetch_tmap(&tmk);
                 prefetch_tmap(&tmv);
                 prefetch_tmap(&tmy);
             }
             mbar_init(mbar + warp, 1);
             fence_mbar_init();
-            if (warp == 0 && bulk) {
-                const uint32_t nb = Cg * 4;
-                const int64_t ch = (int64_t)b * C + c0;
-                mbar_arrive_expect_tx(pbar, (p.state_in ? 5u : 2u) * nb);
-                bulk_load(sw, p.w + c0, nb, pbar);
-                bulk_load(sw + Cg, p.u + c0, nb, pbar);
-                if (p.state_in) {
-                    bulk_load(sw + 2 * Cg, p.state_in + ch, nb, pbar);
-                    bulk_load(sw + 3 * Cg, p.state_in + p.BC + ch, nb, pbar);
-                    bulk_load(sw + 4 * Cg, p.state_in + 2 * p.BC + ch, nb, pbar);
-                }
-            }
-            issue_rows(0);
+            if (warp == 0 && bulk_ok(c0)) issue_params(0, b, c0);
+            issue_rows(0, b, c0);
         }
         __syncwarp();
     }
     // tensor memory after the loads are on their way
     if (warp == 0) tmem_alloc(tslot, (uint32_t)lay.tmem_cols());
-    PairConsts cc;
-    St carry[2];  // the state carried into the current round (warp 1 folds it)
-    if (!bulk) {
-        pair_wu(p.w, p.u, c0 + col, C, cc);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int64_t c = c0 + col + j;
-            carry[j] = (p.state_in && c < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c)
-                                             : empty_state();
-        }
-    }
     // the tensor-memory base is in shared memory, every barrier initialised
     tmem_fence_before_sync();
     __syncthreads();
@@ -372,31 +388,58 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         return tbase + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(s * NW * L + (warp >> 2) * 4 * L);
     };
     bool failed = false;
-    if (bulk) {
-        if (!mbar_wait_bounded(pbar, 0)) {
-            failed = true;
-            if (lane == 0) atomicOr(&g_device_error, kErrTmaWait);
-        }
+
+    // w, u of the current tile (cc) and the state carried into it (carry;
+    // only warp 1 folds it), from parameter slot `slot` (its phase `parity`)
+    // or, for a partial or unaligned slice, from global memory
+    PairConsts cc;
+    St carry[2];
+    auto take_params = [&](int slot, uint32_t parity) {
+        if (bulk_ok(c0)) {
+            if (!failed && !mbar_wait_bounded(pbar + slot, parity)) {
+                failed = true;
+                if (lane == 0) atomicOr(&g_device_error, kErrTmaWait);
+            }
+            const float* sw = reinterpret_cast<const float*>(base + lay.params(slot));
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            cc.w[j] = sw[col + j];
-            cc.u[j] = sw[Cg + col + j];
-            carry[j] = p.state_in ? St{sw[2 * Cg + col + j], sw[3 * Cg + col + j],
-                                       (double)sw[4 * Cg + col + j] * kLog2eD}
-                                  : empty_state();
+            for (int j = 0; j < 2; ++j) {
+                cc.w[j] = sw[col + j];
+                cc.u[j] = sw[Cg + col + j];
+                carry[j] = p.state_in ? St{sw[2 * Cg + col + j], sw[3 * Cg + col + j],
+                                           (double)sw[4 * Cg + col + j] * kLog2eD}
+                                      : empty_state();
+            }
+        } else {
+            pair_wu(p.w, p.u, c0 + col, C, cc);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int64_t c = c0 + col + j;
+                carry[j] = (p.state_in && c < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c)
+                                                 : empty_state();
+            }
         }
-    }
-    pair_derive(cc);
+        pair_derive(cc);
+    };
+    auto put_state_out = [&]() {
+        if (rank == 0 && warp == 1 && p.state_out) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int64_t c = c0 + col + j;
+                if (c < C) store_state_log2(p.state_out, p.BC, (int64_t)b * C + c, carry[j]);
+            }
+        }
+    };
 
     // ---- 1. summary pass of a round: this warp's chunk summary into its
     //         entry of summary slot round & 1 (kMulti) and its stash into
-    //         tensor-memory slot round & 1; then its rows take the next round's
-    auto summary = [&](int round) -> PairRef {
+    //         tensor-memory slot round & 1, once its rows (barrier phase
+    //         `parity`) are in
+    auto summary = [&](int round, uint32_t parity) -> PairRef {
         const int slot = kMulti ? (round & 1) : 0;
         const int n = chunk_len(round, warp);
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;  // segment start
         if constexpr (kTMA) {
-            if (n > 0 && !failed && !mbar_wait_bounded(mbar + warp, (uint32_t)(round & 1))) {
+            if (n > 0 && !failed && !mbar_wait_bounded(mbar + warp, parity)) {
                 failed = true;
                 if (lane == 0) atomicOr(&g_device_error, kErrTmaWait);
             }
@@ -422,22 +465,18 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         const TripleRef sums = triples(base + lay.sums(slot), NW * Cg);
 #pragma unroll
         for (int j = 0; j < 2; ++j) sums.put(warp * Cg + col + j, sum[j]);
-        if constexpr (kTMA && kMulti) {
-            __syncwarp();  // every lane has read the rows
-            if (lane == 0) issue_rows(round + 1);
-        }
         return ref;
     };
 
-    // ---- 2. warp 0, once every warp's summary of the round is in: the
+    // ---- 2. warp 0, once every warp's summary of exchange `it` is in: the
     //         segment aggregate (one round: the chunk summaries joined as a
     //         tree; several rounds: with their exclusive prefix, in place, by
     //         one chain) goes by asynchronous DSMEM stores into slot
-    //         [round % kAS][rank] of every CTA of the cluster, each store
+    //         [it % kAS][rank] of every CTA of the cluster, each store
     //         completing bytes on that CTA's barrier of the slot
-    auto scan_push = [&](int round) {
+    auto scan_push = [&](int round, int it) {
         const TripleRef sums = triples(base + lay.sums(kMulti ? (round & 1) : 0), NW * Cg);
-        const TripleRef agg = triples(base + lay.agg(round % kAS), NC * Cg);
+        const TripleRef agg = triples(base + lay.agg(it % kAS), NC * Cg);
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
         // steps of this CTA's segment (the chunks' lengths follow from it)
         const int rem = (int)max((int64_t)0, min((int64_t)Ts, T - t0));
@@ -459,7 +498,7 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         }
         const int off = rank * Cg + col;
         const uint32_t la = smem_u32(agg.a + off), lb = smem_u32(agg.b + off);
-        const uint32_t lp = smem_u32(agg.p + off), lbar = smem_u32(abar + round % kAS);
+        const uint32_t lp = smem_u32(agg.p + off), lbar = smem_u32(abar + it % kAS);
 #pragma unroll 1
         for (int q = 0; q < NC; ++q) {
             const uint32_t rbar = mapa_u32(lbar, (uint32_t)q);
@@ -469,26 +508,25 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         }
     };
 
-    // ---- 3. warp 1, once the round's aggregates have landed: the state at
-    //         this CTA's segment start (the state carried into the round
-    //         joined with the aggregates of the segments before it) into
-    //         start slot round & 1, and the state carried into the next round
-    //         (joined with all of them).  Only warp 1 holds the carried state.
-    auto fold = [&](int round) {
-        const int as = round % kAS;
+    // ---- 3. warp 1, once the aggregates of exchange `it` have landed: the
+    //         state at this CTA's segment start (the state carried into the
+    //         round joined with the aggregates of the segments before it)
+    //         into start slot round & 1, and the state carried into the next
+    //         round (joined with all of them)
+    auto fold = [&](int round, int it) {
+        const int as = it % kAS;
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
         const TripleRef agg = triples(base + lay.agg(as), NC * Cg);
-        if (!failed && !mbar_wait_cluster_bounded(abar + as, (uint32_t)((round / kAS) & 1))) {
+        if (!failed && !mbar_wait_cluster_bounded(abar + as, (uint32_t)((it / kAS) & 1))) {
             failed = true;
             if (lane == 0) atomicOr(&g_device_error, kErrExchangeWait);
         }
-        // The slot's next use is round + 2.  Every CTA pushes round + 2 after
-        // its CTA barrier of round + 1, which follows its own fold of round
-        // + 1, which waited for this CTA's push of round + 1, issued after
-        // this CTA's barrier of round, which this warp reaches after this
-        // fold: the slot is read before it is overwritten, and re-armed (here)
-        // before it is written.
-        if (lane == 0 && round + kAS < p.rounds) mbar_arrive_expect_tx(abar + as, agg_bytes);
+        // The slot's next use is exchange it + 2.  Every CTA pushes it + 2
+        // after its CTA barrier that follows its own fold of it + 1, which
+        // waited for this CTA's push of it + 1, issued after the barrier
+        // that follows this fold: the slot is read before it is overwritten,
+        // and re-armed (here) before it is written.
+        if (lane == 0 && it + kAS < items) mbar_arrive_expect_tx(abar + as, agg_bytes);
         const int64_t rrem = T - (t0 - (int64_t)rank * Ts);  // steps of the round from segment 0 on
         St P[2];
         switch (NC) {
@@ -528,7 +566,11 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
     };
 
     // ---- 4. every warp: its chunk's outputs from the stash and the state S
-    //         at its start
+    //         at its start.  One round (TMA launch): y is staged in place of v
+    //         and sent out by one TMA store.  Several rounds (the rows already
+    //         hold the next round's): y goes straight from registers, one
+    //         2-channel store a step per lane (C % 4 == 0 with TMA, so a pair
+    //         in range is whole and aligned).
     auto emit = [&](int round, const PairRef& ref, const St (&S)[2]) {
         const int slot = kMulti ? (round & 1) : 0;
         const int n = chunk_len(round, warp);
@@ -536,41 +578,35 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         const int64_t cpair = c0 + col;
         const int64_t row0 = ((int64_t)b * T + t0 + warp * L) * C + cpair;  // k, v, y offset
         const bool ok0 = cpair < C, ok1 = cpair + 1 < C;
-        if constexpr (kTMA && !kMulti) {
-            // one round: y staged in place of k, sent out by one TMA store
-            IO* yr = kr;
-            auto st_one = [=](int s, int j, float y) { yr[s * Cg + col + j] = Io<IO>::from_f(y); };
-            auto st_pair = [=](int s, f2 y) { Pair<IO>::store(yr + s * Cg + col, y); };
-            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
-                                      st_pair, st_one);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                if (n > 0 && !failed) {
-                    tma_store_3d(&tmy, yr, (int)c0, (int)(t0 + warp * L), b);
-                    bulk_commit();
+        IO* yrow = yg + row0;
+        auto out_one = [=](int s, int j, float y) {
+            if (j == 0 ? ok0 : ok1) yrow[(int64_t)s * C + j] = Io<IO>::from_f(y);
+        };
+        if constexpr (kTMA) {
+            if constexpr (!kMulti) {
+                IO* yr = vr;
+                auto st_one = [=](int s, int j, float y) { yr[s * Cg + col + j] = Io<IO>::from_f(y); };
+                auto st_pair = [=](int s, f2 y) { Pair<IO>::store(yr + s * Cg + col, y); };
+                chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
+                                          st_pair, st_one);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (n > 0 && !failed) {
+                        tma_store_3d(&tmy, yr, (int)c0, (int)(t0 + warp * L), b);
+                        bulk_commit();
+                    }
                 }
+                __syncwarp();
+            } else {
+                auto out_pair = [=](int s, f2 y) {
+                    if (ok0) Pair<IO>::store(yrow + (int64_t)s * C, y);
+                };
+                chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
+                                          out_pair, out_one);
             }
-            __syncwarp();
-        } else if constexpr (kTMA) {
-            // several rounds (the rows already hold the next round's): y
-            // straight from registers, one 2-channel store a step per lane
-            // (C % 4 == 0 with TMA, so a pair in range is whole and aligned)
-            IO* yrow = yg + row0;
-            auto out_one = [=](int s, int j, float y) {
-                if (j == 0 ? ok0 : ok1) yrow[(int64_t)s * C + j] = Io<IO>::from_f(y);
-            };
-            auto out_pair = [=](int s, f2 y) {
-                if (ok0) Pair<IO>::store(yrow + (int64_t)s * C, y);
-            };
-            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
-                                      out_pair, out_one);
         } else {
             // element-wise stores (any alignment)
-            IO* yrow = yg + row0;
-            auto out_one = [=](int s, int j, float y) {
-                if (j == 0 ? ok0 : ok1) yrow[(int64_t)s * C + j] = Io<IO>::from_f(y);
-            };
             auto out_pair = [=](int s, f2 y) {
                 if (ok0) yrow[(int64_t)s * C] = Io<IO>::from_f(lo(y));
                 if (ok1) yrow[(int64_t)s * C + 1] = Io<IO>::from_f(hi(y));
@@ -580,23 +616,61 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         }
     };
 
-    PairRef ref_cur = summary(0);
-    __syncthreads();  // every summary of round 0 is in
-    cluster_wait();   // every CTA of the cluster has started
-    if (warp == 0) scan_push(0);
     if constexpr (!kMulti) {
-        // one round (the launch guarantees it); each warp joins the summaries
-        // before its chunk while the aggregates travel
-        St E[2];
-        int nE;
-        chunk_prefix(E, nE);
-        if (warp == 1) fold(0);
-        __syncthreads();  // the segment start state is in place
-        const TripleRef st = triples(base + lay.start(0), Cg);
-        St S[2];
+        // One round per tile; the cluster walks tiles tile, tile + G, ...  A
+        // warp's k rows of the next tile (and warp 0's parameters of it) are
+        // loaded as soon as its summary pass is done, so they land while the
+        // aggregates travel and the outputs go out; its v rows once the TMA
+        // store of y, staged in them, has read them (a TMA store beats one
+        // store a step from registers).  Per tile j (exchange j):
+        //   summary -> barrier A -> warp 0 pushes, every warp joins its chunk
+        //   prefix, warp 1 folds -> barrier B -> outputs.
+        // Slots in use across tiles: parameters and aggregates alternate
+        // (j & 1); the summaries, the stash and the start state are rewritten
+        // only after barrier B of the tile that read them.
+        for (int j = 0; j < items; ++j) {
+            const bool more = j + 1 < items;
+            take_params(j & 1, (uint32_t)((j >> 1) & 1));
+            const PairRef ref = summary(0, (uint32_t)(j & 1));
+            const int nt = tile + G, nb = nt / p.CGB;  // the next tile, if `more`
+            const int64_t nc0 = (int64_t)(nt - nb * p.CGB) * Cg;
+            if (kTMA && more) {
+                __syncwarp();  // every lane has read the rows
+                if (lane == 0) {
+                    if (warp == 0 && bulk_ok(nc0)) issue_params((j + 1) & 1, nb, nc0);
+                    issue_k(0, nb, nc0);
+                }
+            }
+            __syncthreads();  // A: every summary of the tile is in
+            if (j == 0) cluster_wait();  // every CTA of the cluster has started
+            if (warp == 0) scan_push(0, j);
+            St E[2];
+            int nE;
+            chunk_prefix(E, nE);
+            if (warp == 1) {
+                fold(0, j);
+                put_state_out();
+            }
+            __syncthreads();  // B: the segment start state is in place
+            const TripleRef st = triples(base + lay.start(0), Cg);
+            St S[2];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) S[j] = combine(st.get(col + j), E[j], (double)nE * cc.w2[j]);
-        emit(0, ref_cur, S);
+            for (int q = 0; q < 2; ++q) S[q] = combine(st.get(col + q), E[q], (double)nE * cc.w2[q]);
+            emit(0, ref, S);
+            if (kTMA && more) {
+                if (lane == 0) {
+                    bulk_wait_read_all();  // the staged y has been read
+                    issue_v(0, nb, nc0);
+                }
+                __syncwarp();
+            }
+            if (more) {
+                tile += G;
+                b = tile / p.CGB;
+                c0 = (int64_t)(tile - b * p.CGB) * Cg;
+            }
+        }
+        if (kTMA && lane == 0) bulk_wait_read_all();  // staged rows stay valid until read
     } else {
         // Round r + 1's summary pass runs while round r's aggregates are on
         // their way.  One CTA barrier a round (B_r): before it every warp has
@@ -604,33 +678,41 @@ __global__ void __maxnreg__(WKV4_SCAN_MAXNREG)
         // round r, and warp 1 has folded round r; after it warp 0 scans and
         // pushes round r + 1, every warp emits round r, and warp 1 folds round
         // r + 1, whose aggregates have had a whole output pass to arrive.
+        take_params(0, 0);
+        PairRef ref_cur = summary(0, 0);
+        if (kTMA && p.rounds > 1) {
+            __syncwarp();  // every lane has read the rows
+            if (lane == 0) issue_rows(1, b, c0);
+        }
+        __syncthreads();  // every summary of round 0 is in
+        cluster_wait();   // every CTA of the cluster has started
+        if (warp == 0) scan_push(0, 0);
         for (int round = 0; round < p.rounds; ++round) {
             const bool more = round + 1 < p.rounds;
             PairRef ref_next = ref_cur;
-            if (more) ref_next = summary(round + 1);
-            if (round == 0 && warp == 1) fold(0);
+            if (more) {
+                ref_next = summary(round + 1, (uint32_t)((round + 1) & 1));
+                if (kTMA && round + 2 < p.rounds) {
+                    __syncwarp();  // every lane has read the rows
+                    if (lane == 0) issue_rows(round + 2, b, c0);
+                }
+            }
+            if (round == 0 && warp == 1) fold(0, 0);
             __syncthreads();
-            if (more && warp == 0) scan_push(round + 1);
+            if (more && warp == 0) scan_push(round + 1, round + 1);
             St S[2];
             chunk_start(round, S);
             emit(round, ref_cur, S);
-            if (more && warp == 1) fold(round + 1);
+            if (more && warp == 1) fold(round + 1, round + 1);
             ref_cur = ref_next;
         }
+        put_state_out();
     }
-    if (kTMA && !kMulti && lane == 0) bulk_wait_read_all();  // staged rows stay valid until read
 
-    if (rank == 0 && warp == 1 && p.state_out) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int64_t c = c0 + col + j;
-            if (c < C) store_state_log2(p.state_out, p.BC, (int64_t)b * C + c, carry[j]);
-        }
-    }
     // Every warp's tensor-memory accesses have completed (each load and each
     // store pass ends in its wait); release the columns.  No cluster barrier
-    // is needed before leaving: peers only write into this CTA's shared
-    // memory before a round's cluster barrier, and read only their own.
+    // is needed before leaving: every aggregate pushed into this CTA has
+    // landed (its fold waited for it), and peers read only their own memory.
     tmem_fence_before_sync();
     __syncthreads();
     tmem_fence_after_sync();
