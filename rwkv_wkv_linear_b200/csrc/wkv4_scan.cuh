@@ -79,8 +79,11 @@ struct ScanLayout {
     __host__ __device__ size_t sums(int slot) const {  // [kSlots][nw][Cg] x 16 B
         return 2 * tile() + (size_t)slot * nw * kCg * 16;
     }
+    // one round: the exclusive prefixes of the chunk summaries, [nw][Cg] x 16 B
+    // (several rounds scan the summaries in place)
+    __host__ __device__ size_t pre() const { return sums(kSlots); }
     __host__ __device__ size_t start(int slot) const {  // [kSlots][Cg] x 16 B
-        return sums(kSlots) + (size_t)slot * kCg * 16;
+        return pre() + (kMulti ? 0 : (size_t)nw * kCg * 16) + (size_t)slot * kCg * 16;
     }
     __host__ __device__ size_t agg(int slot) const {  // [kAggSlots][nc][Cg] x 16 B
         return start(kSlots) + (size_t)slot * nc * kCg * 16;
@@ -172,51 +175,13 @@ __device__ __forceinline__ void tree_range(const TripleRef& t, int col, int lo, 
     }
 }
 
-// Stretches 0 .. m - 1 of N joined (m warp-uniform, 0 <= m < N): the state
-// contribution before stretch m (the empty state for m = 0), spanning npre.
-template <int N, typename Len>
-__device__ __forceinline__ void tree_prefix(const TripleRef& t, int col, int m, Len len,
-                                            const PairConsts& cc, St (&pre)[2], int& npre) {
-    pre[0] = pre[1] = empty_state();
-    npre = 0;
-    int lo = 0;
-    auto add = [&](const St (&y)[2], int ny) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) pre[j] = combine(pre[j], y[j], (double)ny * cc.w2[j]);
-        npre += ny;
-    };
-    if constexpr (N >= 8) {
-        if (m & 4) {
-            tree_range<4>(t, col, 0, len, cc, pre, npre);
-            lo = 4;
-        }
-    }
-    if constexpr (N >= 4) {
-        if (m & 2) {
-            St y[2];
-            int ny;
-            tree_range<2>(t, col, lo, len, cc, y, ny);
-            add(y, ny);
-            lo += 2;
-        }
-    }
-    if constexpr (N >= 2) {
-        if (m & 1) {
-            St y[2];
-            int ny;
-            tree_range<1>(t, col, lo, len, cc, y, ny);
-            add(y, ny);
-        }
-    }
-}
-
-// Warp 0: exclusive prefix of the NW chunk summaries of a segment (in
-// place: entry q becomes the state before chunk q) and the segment aggregate
-// in acc.  All summaries are read before the chain starts; chunk q spans
-// clamp(rem - q L, 0, L) steps.
+// Exclusive prefix of the NW chunk summaries of a segment into `out` (entry
+// q becomes the state before chunk q; `out` may be `sums` itself) and the
+// segment aggregate in acc.  All summaries are read before the chain starts;
+// chunk q spans clamp(rem - q L, 0, L) steps.
 template <int NW, int L>
-__device__ __forceinline__ void scan_chunks(const TripleRef& sums, int col, int rem,
-                                            const PairConsts& cc, St (&acc)[2]) {
+__device__ __forceinline__ void scan_chunks(const TripleRef& sums, const TripleRef& out, int col,
+                                            int rem, const PairConsts& cc, St (&acc)[2]) {
     constexpr int Cg = 64;
     St x[NW][2];
 #pragma unroll
@@ -229,7 +194,7 @@ __device__ __forceinline__ void scan_chunks(const TripleRef& sums, int col, int 
         const double nq = (double)max(0, min(L, rem - q * L));
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-            sums.put(q * Cg + col + j, acc[j]);
+            out.put(q * Cg + col + j, acc[j]);
             acc[j] = combine(acc[j], x[q][j], nq * cc.w2[j]);
         }
     }
@@ -483,9 +448,9 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
         St acc[2];
         if constexpr (kMulti) {
             if (NW == 8) {
-                scan_chunks<8, L>(sums, col, rem, cc, acc);
+                scan_chunks<8, L>(sums, sums, col, rem, cc, acc);
             } else {
-                scan_chunks<4, L>(sums, col, rem, cc, acc);
+                scan_chunks<4, L>(sums, sums, col, rem, cc, acc);
             }
         } else {
             auto clen = [=](int q) { return max(0, min(L, rem - q * L)); };
@@ -552,16 +517,18 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
             S[j] = combine(st.get(col + j), sums.get(warp * Cg + col + j), (double)(warp * L) * cc.w2[j]);
     };
 
-    // ---- one round, every warp, once every summary is in: the summaries of
-    //      the chunks before its own joined (E, spanning nE steps)
-    auto chunk_prefix = [&](St (&E)[2], int& nE) {
+    // ---- one round, warp 2, once every summary is in: the exclusive prefix
+    //      of the chunk summaries (one chain) into the prefix array, while
+    //      warp 0 pushes and warp 1 folds
+    auto chunk_prefixes = [&]() {
         const TripleRef sums = triples(base + lay.sums(0), NW * Cg);
+        const TripleRef pre = triples(base + lay.pre(), NW * Cg);
         const int rem = (int)max((int64_t)0, min((int64_t)Ts, T - (int64_t)rank * Ts));
-        auto clen = [=](int q) { return max(0, min(L, rem - q * L)); };
+        St acc[2];
         if (NW == 8) {
-            tree_prefix<8>(sums, col, warp, clen, cc, E, nE);
+            scan_chunks<8, L>(sums, pre, col, rem, cc, acc);
         } else {
-            tree_prefix<4>(sums, col, warp, clen, cc, E, nE);
+            scan_chunks<4, L>(sums, pre, col, rem, cc, acc);
         }
     };
 
@@ -623,8 +590,8 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
         // aggregates travel and the outputs go out; its v rows once the TMA
         // store of y, staged in them, has read them (a TMA store beats one
         // store a step from registers).  Per tile j (exchange j):
-        //   summary -> barrier A -> warp 0 pushes, every warp joins its chunk
-        //   prefix, warp 1 folds -> barrier B -> outputs.
+        //   summary -> barrier A -> warp 0 pushes, warp 2 scans the chunk
+        //   prefixes, warp 1 folds -> barrier B -> outputs.
         // Slots in use across tiles: parameters and aggregates alternate
         // (j & 1); the summaries, the stash and the start state are rewritten
         // only after barrier B of the tile that read them.
@@ -644,18 +611,18 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
             __syncthreads();  // A: every summary of the tile is in
             if (j == 0) cluster_wait();  // every CTA of the cluster has started
             if (warp == 0) scan_push(0, j);
-            St E[2];
-            int nE;
-            chunk_prefix(E, nE);
+            if (warp == 2) chunk_prefixes();
             if (warp == 1) {
                 fold(0, j);
                 put_state_out();
             }
-            __syncthreads();  // B: the segment start state is in place
+            __syncthreads();  // B: the segment start state and the chunk prefixes are in place
             const TripleRef st = triples(base + lay.start(0), Cg);
+            const TripleRef pre = triples(base + lay.pre(), NW * Cg);
             St S[2];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) S[q] = combine(st.get(col + q), E[q], (double)nE * cc.w2[q]);
+            for (int q = 0; q < 2; ++q)
+                S[q] = combine(st.get(col + q), pre.get(warp * Cg + col + q), (double)(warp * L) * cc.w2[q]);
             emit(0, ref, S);
             if (kTMA && more) {
                 if (lane == 0) {
