@@ -21,6 +21,9 @@ loop of wkv4_decode_step calls over one fp32 state updated in place, captured
 as one CUDA graph; each call's k, v come from a pool of seeded inputs that
 rotates over more than 3x the L2 cache.  The state (12 B a channel) stays
 L2-resident across calls by design, so the line's GB/s is effective.
+``--workload decode_slots_b256`` is the slot-indexed decode: each call serves
+256 rows from a pool of 1024 states (wkv4_decode_step_slots), its slot ids
+drawn per call.
 
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead
 (rank 0 only; other ranks exit).
@@ -395,6 +398,27 @@ def run_reference(args):
 
     wl = synth.workload(args.workload)
     config = {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C, "io_dtype": wl.dtype}
+    if wl.slots:
+        # the oracle's slot-indexed decode over a bounded sample of the calls
+        for _ in range(args.warmup):
+            cpu_baseline_slots(wl)
+        t0 = time.perf_counter()
+        base = None
+        for _ in range(args.steps):
+            base = cpu_baseline_slots(wl)
+        dt = time.perf_counter() - t0
+        config.update(calls=wl.steps, slots=wl.slots)
+        line = {
+            "impl": "reference", "metric": METRIC, "value": base["value"], "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     if wl.T == 1:
         # a decode loop over one state is a forward over the calls' time axis
         wl, x = _decode_as_forward(wl)
@@ -481,14 +505,22 @@ def run_decode(args):
         ks.append(k.to(dev))
         vs.append(v.to(dev))
     ys = [torch.empty_like(ks[0]) for _ in range(pool)]
-    state = synth.zero_state(wl.B, wl.C).to(dev)
+    slots = wl.slots > 0
+    state = synth.zero_state(wl.slots if slots else wl.B, wl.C).to(dev)
+    ids = [synth.decode_slot_ids(wl, s_).to(dev) for s_ in range(pool)] if slots else None
     stream = torch.cuda.Stream(device=dev)
     n = wl.steps
+
+    def call(kd, vd, yd, j):
+        if slots:
+            wkv4.decode_step_slots(kd, vd, w, u, state, ids[j], y=yd, stream=stream)
+        else:
+            wkv4.decode_step(kd, vd, w, u, state, y=yd, stream=stream)
 
     def loop():
         for s_ in range(n):
             j = s_ % pool
-            wkv4.decode_step(ks[j], vs[j], w, u, state, y=ys[j], stream=stream)
+            call(ks[j], vs[j], ys[j], j)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -522,22 +554,28 @@ def run_decode(args):
     clocks.stop()
     ms = max_over_ranks(start.elapsed_time(end), dev)
     if wkv4.device_error() != 0:
-        raise RuntimeError("device-side wait ran out during the timed region")
+        raise RuntimeError("device-side error during the timed region")
 
-    # end to end through the C ABI: every call's k, v from pinned host memory,
-    # its y back to the host
+    # end to end through the C ABI: every call's k, v (and slot ids) from
+    # pinned host memory, its y back to the host
     e2e = None
     if not args.no_e2e:
         n_e2e = max(1, args.e2e_steps)
         kh = [ks[j % pool].cpu().pin_memory() for j in range(min(pool, n_e2e))]
         vh = [vs[j % pool].cpu().pin_memory() for j in range(min(pool, n_e2e))]
+        ih = [ids[j % pool].cpu().pin_memory() for j in range(min(pool, n_e2e))] if slots else None
         yh = torch.empty_like(kh[0]).pin_memory()
         kd, vd, yd = ks[0], vs[0], ys[0]
+        idd = torch.empty_like(ids[0]) if slots else None
 
         def e2e_call(j):
             kd.copy_(kh[j % len(kh)], non_blocking=True)
             vd.copy_(vh[j % len(vh)], non_blocking=True)
-            wkv4.decode_step(kd, vd, w, u, state, y=yd, stream=stream)
+            if slots:
+                idd.copy_(ih[j % len(ih)], non_blocking=True)
+                wkv4.decode_step_slots(kd, vd, w, u, state, idd, y=yd, stream=stream)
+            else:
+                wkv4.decode_step(kd, vd, w, u, state, y=yd, stream=stream)
             yh.copy_(yd, non_blocking=True)
 
         with torch.cuda.stream(stream):
@@ -555,13 +593,15 @@ def run_decode(args):
         torch.cuda.synchronize()
         t2_ms = max_over_ranks(s2.elapsed_time(e2), dev)
         e2e = {"value": job_throughput(wl.B * wl.C, n_e2e, world, t2_ms), "unit": UNIT,
-               "h2d_bytes_per_step": call_io, "d2h_bytes_per_step": io_bytes(wl),
+               "h2d_bytes_per_step": call_io + (4 * wl.B if slots else 0),
+               "d2h_bytes_per_step": io_bytes(wl),
                "steps": n_e2e, "step": "one decode call"}
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
         calls = K * n
-        call_bytes = 3 * io_bytes(wl) + 24 * wl.B * wl.C  # k, v, y + state read and written
+        # k, v, y + state read and written (+ the slot ids)
+        call_bytes = 3 * io_bytes(wl) + 24 * wl.B * wl.C + (4 * wl.B if slots else 0)
         achieved = call_bytes / (ms / 1e3 / calls) / 1e9
         line = {
             "metric": METRIC,
@@ -577,10 +617,14 @@ def run_decode(args):
             "dtype": "f32",
             "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C, "calls": n,
-                       "io_dtype": wl.dtype, "state": "fp32, in place, zero at the start",
+                       "io_dtype": wl.dtype,
+                       "state": (f"fp32 pool of {wl.slots} states, rows named by per-call slot ids, "
+                                 "in place, zero at the start") if slots else
+                                "fp32, in place, zero at the start",
                        "global_batch": wl.B * world, "seq_len": n,
                        "parallelism": f"independent sequences per rank (x{world})",
-                       "step": f"one decode loop of {n} wkv4_decode_step calls",
+                       "step": f"one decode loop of {n} "
+                               f"{'wkv4_decode_step_slots' if slots else 'wkv4_decode_step'} calls",
                        "l2": f"k, v rotate over {pool} seeded call inputs "
                              f"({pool * call_io / 1e6:.0f} MB > 3x L2); the state is L2-resident",
                        "launch": f"one CUDA graph of {n} calls per step, {K} replays"},
@@ -593,7 +637,7 @@ def run_decode(args):
             "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline_decode(wl)
+            line["cpu_baseline"] = cpu_baseline_slots(wl) if slots else cpu_baseline_decode(wl)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -635,6 +679,45 @@ def cpu_baseline_decode(wl):
             "sample": f"batch rows 0..{ws.B - 1} of {wl.B} x calls 0..{ws.T - 1} of {wl.steps}, "
                       f"C={wl.C} ({ws.channel_steps} channel-steps) x {reps} passes, fp64 C "
                       f"recurrence, {cores} threads over channels"}
+
+
+def _slots_sample(wl, rows: int = 16, pool: int = 64, calls: int = 32):
+    """A bounded sample of a slot-indexed decode workload for the oracle: the
+    first `rows` rows of each of the first `calls` calls, their ids folded
+    into a pool of `pool` states (ids mod pool, made distinct per call)."""
+    import numpy as np
+    from rwkv_wkv_linear_b200 import synth
+    w, u = synth.decode_params(wl)
+    calls = min(calls, wl.steps)
+    steps = []
+    for s_ in range(calls):
+        k, v = synth.decode_step_inputs(wl, s_)
+        ids = synth.decode_slot_ids(wl, s_).numpy()[:rows] % pool
+        _, first = np.unique(ids, return_index=True)  # one row per slot within a call
+        keep = np.sort(first)
+        steps.append((k[:rows][keep], v[:rows][keep], ids[keep]))
+    return w, u, steps, pool
+
+
+def cpu_baseline_slots(wl):
+    """The oracle's slot-indexed decode over a bounded sample (_slots_sample)."""
+    import numpy as np
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    w, u, steps, pool = _slots_sample(wl)
+    n_ch = sum(len(ids) for _, _, ids in steps) * wl.C
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        st = oracle.empty_state(pool, wl.C)
+        for k, v, ids in steps:
+            _, st, _ = oracle.decode_slots(k, v, w, u, st, ids)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if reps >= 3 and dt > 1.0 or dt > 20.0:
+            break
+    return {"value": n_ch * reps / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{len(steps)} calls x up to 16 rows of {wl.B} from a pool of {pool} states, "
+                      f"C={wl.C} ({n_ch} channel-steps) x {reps} passes, fp64 C recurrence per row"}
 
 
 def main():

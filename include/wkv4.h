@@ -65,7 +65,8 @@ enum {
     WKV4_ERR_ALIAS = -3,   /* y or the output state overlaps an input it must not */
     WKV4_ERR_CUDA = -4,    /* a CUDA runtime call or kernel launch failed */
     WKV4_ERR_TIMEOUT = -5, /* a bounded device-side wait ran out (see wkv4_device_error) */
-    WKV4_ERR_VARIANT = -7  /* unknown kernel variant */
+    WKV4_ERR_VARIANT = -7, /* unknown kernel variant */
+    WKV4_ERR_SLOT = -8     /* a decode row named a state slot outside the pool (see wkv4_device_error) */
 };
 
 /*
@@ -121,12 +122,41 @@ WKV4_API int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float*
                      const void* v, float* state, void* y, wkv4_stream_t stream, int dtype);
 
 /*
+ * One decode step (T = 1) for B sequences whose states live in a pool of S
+ * slots: row b of k, v and y steps the state in slot slot_ids[b], in place.
+ * The RNN state as a first-class object that the caller keeps per
+ * conversation ("An RNN that claims to match transformers, now in chatbot
+ * form", sections "The interesting bit" and "Caveats"), for many
+ * conversations served together.
+ *   w, u        [C] fp32.
+ *   k, v        [B][C] in `dtype`.
+ *   state_pool  [3][S][C] fp32 (planes numerator, denominator, max); the rows
+ *               slot_ids[b] are read and overwritten, every other row is left
+ *               as it is.
+ *   slot_ids    [B] int32 in device memory, each in [0, S), all distinct
+ *               (repeated ids make their rows race on one slot: undefined).
+ *               A row whose id is outside [0, S) touches neither the pool
+ *               nor its row of y, and sets bit 8 of the device error word
+ *               (wkv4_device_error then returns WKV4_ERR_SLOT).
+ *   y           [B][C] in `dtype`.
+ * y must not overlap k, v, w, u, the pool or slot_ids, and the pool must not
+ * overlap k, v, w, u or slot_ids: WKV4_ERR_ALIAS.  S < 0: WKV4_ERR_ARG.
+ * Per row, equal bit for bit to wkv4_decode_step on that row's state.  The
+ * call allocates no memory.
+ */
+WKV4_API int wkv4_decode_step_slots(int64_t B, int64_t C, int64_t S, const float* w, const float* u,
+                                    const void* k, const void* v, float* state_pool,
+                                    const int32_t* slot_ids, void* y, wkv4_stream_t stream,
+                                    int dtype);
+
+/*
  * Device-side error word of the current device (bit 1: a bounded wait for a
  * TMA copy ran out; bit 2: a bounded wait for a cluster peer's partial state
- * ran out).  Synchronises the device, reads the word, and clears it
- * when `reset` is non-zero.  Returns WKV4_OK when the
- * word is zero, WKV4_ERR_TIMEOUT when a wait ran out, WKV4_ERR_CUDA when the
- * read itself failed.
+ * ran out; bit 8: a slot-indexed decode row named a slot outside its pool).
+ * Synchronises the device, reads the word, and clears it when `reset` is
+ * non-zero.  Returns WKV4_OK when the word is zero, WKV4_ERR_TIMEOUT when a
+ * wait ran out, else WKV4_ERR_SLOT when a slot id was out of range,
+ * WKV4_ERR_CUDA when the read itself failed.
  */
 WKV4_API int wkv4_device_error(int reset);
 

@@ -6,6 +6,8 @@ and imports nothing from it.
 
 * ``forward``       -- fp64 max-trick recurrence in plain C (``wkv4_oracle.c``).
 * ``decode``        -- repeated T=1 forward calls with the state carried in place.
+* ``decode_slots``  -- one T=1 step per batch row on the state slot the row names
+                       in a pool of states (gather, step, scatter).
 * ``brute``         -- the closed-form sums evaluated literally in 50-digit
                        arithmetic (``oracle/brute.py``), for tiny inputs.
 
@@ -94,6 +96,38 @@ def decode(k, v, w, u, state):
     k, v = _f64(k), _f64(v)
     y, s = forward(k[:, None, :], v[:, None, :], w, u, state)
     return y[:, 0, :], s
+
+
+def decode_slots(k, v, w, u, pool, slot_ids):
+    """One T=1 step for each batch row b on pool row slot_ids[b].
+
+    The RNN state as a first-class object the caller keeps per conversation
+    ("An RNN that claims to match transformers, now in chatbot form", sections
+    "The interesting bit" and "Caveats"), for many conversations at once:
+    k, v [B, C]; pool [3, S, C]; slot_ids [B] integers.  Row b gathers its
+    state from pool[:, slot_ids[b], :], takes the step of ``decode`` and
+    scatters the new state back; a row whose id is outside [0, S) is skipped
+    (its y row is NaN, the pool is not touched).  Returns (y [B, C], new pool
+    [3, S, C], number of skipped rows) as fp64 numpy arrays.
+    """
+    k, v = _f64(k), _f64(v)
+    pool = _f64(pool).copy()
+    ids = np.asarray(slot_ids.detach().cpu() if hasattr(slot_ids, "detach") else slot_ids,
+                     dtype=np.int64)
+    B, C = k.shape
+    S = pool.shape[1]
+    assert pool.shape == (3, S, C) and ids.shape == (B,)
+    y = np.full((B, C), np.nan)
+    skipped = 0
+    for b in range(B):
+        s = int(ids[b])
+        if s < 0 or s >= S:
+            skipped += 1
+            continue
+        yb, sb = decode(k[b:b + 1], v[b:b + 1], w, u, pool[:, s:s + 1, :])
+        y[b] = yb[0]
+        pool[:, s, :] = sb[:, 0, :]
+    return y, pool, skipped
 
 
 def empty_state(B: int, C: int) -> np.ndarray:

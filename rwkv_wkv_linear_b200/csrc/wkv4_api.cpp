@@ -179,13 +179,36 @@ int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float* u, const
     return cuda_status(wkv4::launch_decode(a));
 }
 
+int wkv4_decode_step_slots(int64_t B, int64_t C, int64_t S, const float* w, const float* u,
+                           const void* k, const void* v, float* state_pool,
+                           const int32_t* slot_ids, void* y, wkv4_stream_t stream, int dtype) {
+    int rc = check_common(B, 1, C, dtype);
+    if (rc != WKV4_OK) return rc;
+    if (S < 0) return WKV4_ERR_ARG;
+    if (B == 0 || C == 0) return WKV4_OK;
+    if (!w || !u || !k || !v || !y || !state_pool || !slot_ids) return WKV4_ERR_ARG;
+    const size_t es = wkv4::dtype_size(dtype);
+    const uint64_t io = (uint64_t)B * C * es;
+    const Range ry = range_of(y, io), rk = range_of(k, io), rv = range_of(v, io);
+    const Range rw = range_of(w, C * 4), ru = range_of(u, C * 4);
+    const Range rp = range_of(state_pool, (uint64_t)3 * S * C * 4), rs = range_of(slot_ids, B * 4);
+    if (overlap(ry, rk) || overlap(ry, rv) || overlap(ry, rw) || overlap(ry, ru) || overlap(ry, rp) ||
+        overlap(ry, rs))
+        return WKV4_ERR_ALIAS;
+    if (overlap(rp, rk) || overlap(rp, rv) || overlap(rp, rw) || overlap(rp, ru) || overlap(rp, rs))
+        return WKV4_ERR_ALIAS;
+    FwdArgs a{B, 1, C, w, u, k, v, state_pool, y, state_pool, dtype, (cudaStream_t)stream};
+    return cuda_status(wkv4::launch_decode_slots(a, slot_ids, S));
+}
+
 int wkv4_device_error(int reset) {
     unsigned bits = 0;
     if (wkv4::read_device_error(&bits, reset != 0) != cudaSuccess) {
         cudaGetLastError();
         return WKV4_ERR_CUDA;
     }
-    return bits ? WKV4_ERR_TIMEOUT : WKV4_OK;
+    if (bits & (wkv4::kErrTmaWait | wkv4::kErrExchangeWait)) return WKV4_ERR_TIMEOUT;
+    return bits ? WKV4_ERR_SLOT : WKV4_OK;
 }
 
 const char* wkv4_status_string(int status) {
@@ -197,6 +220,7 @@ const char* wkv4_status_string(int status) {
         case WKV4_ERR_CUDA: return "CUDA runtime error";
         case WKV4_ERR_TIMEOUT: return "a bounded device-side wait ran out";
         case WKV4_ERR_VARIANT: return "unknown kernel variant";
+        case WKV4_ERR_SLOT: return "a decode row named a state slot outside the pool";
         default: return "unknown status";
     }
 }

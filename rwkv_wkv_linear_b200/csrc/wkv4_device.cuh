@@ -29,6 +29,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "wkv4_internal.h"  // device error word bits
+
 namespace wkv4 {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -42,9 +44,6 @@ constexpr float kFastStateLift = 44.f;   // carried state's max above the chunk'
 constexpr float kFastMaxU = 44.f;
 constexpr float kFastMaxW = 0.35f;
 
-// device error word bits
-constexpr unsigned kErrTmaWait = 2u;       // a TMA copy did not land in time
-constexpr unsigned kErrExchangeWait = 4u;  // a cluster peer's aggregate did not land in time
 
 
 // A = a 2^p, D = b 2^p.  The max p is carried in fp64 inside the kernels, so

@@ -9,6 +9,11 @@
 
 namespace wkv4 {
 
+// Bits of the device error word (set by the kernels, read by wkv4_device_error).
+constexpr unsigned kErrTmaWait = 2u;       // a TMA copy did not land in time
+constexpr unsigned kErrExchangeWait = 4u;  // a cluster peer's aggregate did not land in time
+constexpr unsigned kErrSlot = 8u;          // a slot-indexed decode row named a slot outside the pool
+
 struct FwdArgs {
     int64_t B, T, C;
     const float* w;
@@ -44,6 +49,8 @@ cudaError_t launch_scan(const FwdArgs& a, bool tma, EncodeFn encode);
 cudaError_t launch_seq(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv);
 cudaError_t launch_step(const FwdArgs& a);     // exact per-step kernel, any T >= 1
 cudaError_t launch_decode(const FwdArgs& a);   // T == 1, vectorised when aligned
+// T == 1 over rows slots[b] of a state pool of S rows (a.state_in == a.state_out == the pool)
+cudaError_t launch_decode_slots(const FwdArgs& a, const int32_t* slots, int64_t S);
 cudaError_t launch_copy_state(const FwdArgs& a);  // T == 0
 
 // Device error word of the current device (synchronous read; optional reset).

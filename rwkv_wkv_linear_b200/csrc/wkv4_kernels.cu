@@ -412,6 +412,33 @@ cudaError_t launch_decode(const FwdArgs& a) {
     return cudaGetLastError();
 }
 
+cudaError_t launch_decode_slots(const FwdArgs& a, const int32_t* slots, int64_t S) {
+    constexpr int V = 4;
+    const size_t es = dtype_size(a.dtype);
+    const bool vec = (a.C % V == 0) && aligned(a.k, V * es) && aligned(a.v, V * es) &&
+                     aligned(a.y, V * es) && aligned(a.w, 16) && aligned(a.u, 16) &&
+                     aligned(a.state_in, 16);
+    StepParams p = step_params(a);
+    p.slots = slots;
+    p.S = S;
+    const int64_t threads = vec ? a.B * a.C / V : a.B * a.C;
+    const unsigned grid = (unsigned)((threads + 255) / 256);
+    if (vec) {
+        switch (a.dtype) {
+            case WKV4_F32: wkv4_decode_kernel<float, V, true><<<grid, 256, 0, a.stream>>>(p); break;
+            case WKV4_F16: wkv4_decode_kernel<__half, V, true><<<grid, 256, 0, a.stream>>>(p); break;
+            default: wkv4_decode_kernel<__nv_bfloat16, V, true><<<grid, 256, 0, a.stream>>>(p); break;
+        }
+    } else {
+        switch (a.dtype) {
+            case WKV4_F32: wkv4_decode_kernel<float, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
+            case WKV4_F16: wkv4_decode_kernel<__half, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
+            default: wkv4_decode_kernel<__nv_bfloat16, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
+        }
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_copy_state(const FwdArgs& a) {
     const int64_t BC = a.B * a.C;
     if (!a.state_out || BC == 0) return cudaSuccess;

@@ -3,7 +3,9 @@
 //   wkv4_step_kernel    one thread per channel, any T (the recurrence as the
 //                       pages state it, step after step).
 //   wkv4_decode_kernel  T = 1 with V channels per thread and vector accesses;
-//                       the state may be updated in place (RNN mode).
+//                       the state may be updated in place (RNN mode); with
+//                       kSlots, row b's state is row slots[b] of a pool of
+//                       S rows (state_in == state_out == the pool).
 //   wkv4_copy_state_kernel  T = 0: state_out <- state_in (or the empty state).
 #pragma once
 
@@ -20,6 +22,8 @@ struct StepParams {
     const float* state_in;
     void* y;
     float* state_out;
+    const int32_t* slots;  // decode from a state pool: row b uses pool row slots[b]
+    int64_t S;             // pool rows
 };
 
 template <typename IO>
@@ -44,7 +48,7 @@ __global__ void __launch_bounds__(256) wkv4_step_kernel(const StepParams p) {
 
 // The caller checks that C % V == 0 and every pointer is aligned to its
 // vector width.
-template <typename IO, int V>
+template <typename IO, int V, bool kSlots = false>
 __global__ void __launch_bounds__(256) wkv4_decode_kernel(const StepParams p) {
     const int64_t BC = p.B * p.C;
     const int64_t ch = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
@@ -55,10 +59,23 @@ __global__ void __launch_bounds__(256) wkv4_decode_kernel(const StepParams p) {
     load_vec<IO, V>(static_cast<const IO*>(p.v) + ch, vv);
     load_vec<float, V>(p.w + c, w);
     load_vec<float, V>(p.u + c, u);
+    // state plane stride and this thread's offset in a plane (with kSlots the
+    // row's slot, read while the loads above are in flight)
+    int64_t SC = BC, sch = ch;
+    if constexpr (kSlots) {
+        const int64_t b = ch / p.C;
+        const int64_t slot = p.slots[b];
+        if (slot < 0 || slot >= p.S) {
+            if (c == 0) atomicOr(&g_device_error, kErrSlot);
+            return;
+        }
+        SC = p.S * p.C;
+        sch = slot * p.C + c;
+    }
     if (p.state_in) {
-        load_vec<float, V>(p.state_in + ch, a);
-        load_vec<float, V>(p.state_in + BC + ch, bb);
-        load_vec<float, V>(p.state_in + 2 * BC + ch, pp);
+        load_vec<float, V>(p.state_in + sch, a);
+        load_vec<float, V>(p.state_in + SC + sch, bb);
+        load_vec<float, V>(p.state_in + 2 * SC + sch, pp);
     } else {
 #pragma unroll
         for (int j = 0; j < V; ++j) {
@@ -79,9 +96,9 @@ __global__ void __launch_bounds__(256) wkv4_decode_kernel(const StepParams p) {
     }
     store_vec<IO, V>(static_cast<IO*>(p.y) + ch, yy);
     if (p.state_out) {
-        store_vec<float, V>(p.state_out + ch, a);
-        store_vec<float, V>(p.state_out + BC + ch, bb);
-        store_vec<float, V>(p.state_out + 2 * BC + ch, pp);
+        store_vec<float, V>(p.state_out + sch, a);
+        store_vec<float, V>(p.state_out + SC + sch, bb);
+        store_vec<float, V>(p.state_out + 2 * SC + sch, pp);
     }
 }
 

@@ -13,6 +13,8 @@ Workloads (sizes of the RWKV-4 models the pages discuss):
 * ``rwkv4_14b_prefill``    B=4,  T=1024,  C=5120, bf16 I/O, zero state
   (d_model 5120 and 1K context of "RWKV-4 14B", "Every architecture field").
 * ``decode_b256``          B=256, C=5120, T=1 per call for 1024 calls, bf16.
+* ``decode_slots_b256``    the same calls, each serving 256 of a pool of 1024
+  conversation states (slot-indexed decode; ids drawn per call).
 * ``long_t65536``          B=1,  T=65536, C=2048, fp32 I/O, 0.1% of k set to +30.
 
 Recipe (the same for every workload; knobs per workload below):
@@ -27,7 +29,8 @@ Recipe (the same for every workload; knobs per workload below):
 * Spikes: exactly ``round(frac * B*T*C)`` distinct flat positions of k, drawn
   without replacement, are *set* to the spike value.
 * Decode draws w, u from ``default_rng(seed)`` and each call's k, v from
-  ``default_rng([seed, step])``.
+  ``default_rng([seed, step])``; a slot-indexed decode call's ids are the first
+  B of a permutation of the pool drawn from ``default_rng([seed, step, 1])``.
 """
 
 from __future__ import annotations
@@ -58,6 +61,7 @@ class Workload:
     spike_frac: float = 0.0
     spike_value: float = 30.0
     steps: int = 1                 # decode workloads: number of T=1 calls
+    slots: int = 0                 # slot-indexed decode: states in the pool (0: one per row)
 
     @property
     def channel_steps(self) -> int:
@@ -79,6 +83,8 @@ WORKLOADS = {
                                   seed=2, k_var=2.0),
     "decode_b256": Workload("decode_b256", B=256, T=1, C=5120, dtype="bf16", seed=3,
                             steps=1024),
+    "decode_slots_b256": Workload("decode_slots_b256", B=256, T=1, C=5120, dtype="bf16", seed=3,
+                                  steps=1024, slots=1024),
     "long_t65536": Workload("long_t65536", B=1, T=65536, C=2048, dtype="f32", seed=4,
                             k_var=4.0, td_range=(-8.0, 2.0), u_range=(-3.0, 3.0),
                             spike_frac=0.001, spike_value=30.0),
@@ -139,6 +145,12 @@ def decode_step_inputs(wl: Workload, step: int):
     k = rng.standard_normal(shape) * math.sqrt(wl.k_var)
     v = rng.standard_normal(shape) * math.sqrt(wl.v_var)
     return _to_io(k, wl.dtype), _to_io(v, wl.dtype)
+
+
+def decode_slot_ids(wl: Workload, step: int) -> torch.Tensor:
+    """int32 [B]: the distinct pool slots that decode call ``step`` serves."""
+    rng = np.random.default_rng([wl.seed, step, 1])
+    return torch.from_numpy(rng.permutation(wl.slots)[:wl.B].astype(np.int32))
 
 
 def custom(B: int, T: int, C: int, dtype: str = "f32", seed: int = 0, **kw) -> dict:

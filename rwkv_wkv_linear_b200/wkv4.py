@@ -22,12 +22,12 @@ F32, F16, BF16 = 0, 1, 2
 KERNEL_AUTO, KERNEL_SEQ, KERNEL_SCAN, KERNEL_SCAN_LDG, KERNEL_STEP = 0, 1, 2, 3, 4
 
 STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_DTYPE", -3: "ERR_ALIAS", -4: "ERR_CUDA",
-          -5: "ERR_TIMEOUT", -7: "ERR_VARIANT"}
+          -5: "ERR_TIMEOUT", -7: "ERR_VARIANT", -8: "ERR_SLOT"}
 
 _DTYPES = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
 
-EXPORTS = ("wkv4_forward", "wkv4_forward_variant", "wkv4_decode_step", "wkv4_device_error",
-           "wkv4_status_string", "wkv4_version")
+EXPORTS = ("wkv4_decode_step", "wkv4_decode_step_slots", "wkv4_device_error", "wkv4_forward",
+           "wkv4_forward_variant", "wkv4_status_string", "wkv4_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -56,6 +56,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.wkv4_forward_variant.restype = i32
             lib.wkv4_decode_step.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp, vp, i32]
             lib.wkv4_decode_step.restype = i32
+            lib.wkv4_decode_step_slots.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32]
+            lib.wkv4_decode_step_slots.restype = i32
             lib.wkv4_device_error.argtypes = [i32]
             lib.wkv4_device_error.restype = i32
             lib.wkv4_status_string.argtypes = [i32]
@@ -157,6 +159,38 @@ def decode_step(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tens
                                  _stream(stream), dt)
     if rc != 0:
         raise Wkv4Error(rc, "wkv4_decode_step")
+    return y
+
+
+def decode_step_slots(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
+                      state_pool: torch.Tensor, slot_ids: torch.Tensor, *,
+                      y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """wkv4_decode_step_slots: k, v [B, C]; state_pool [3, S, C] fp32 whose rows
+    slot_ids [B] (int32, distinct, in [0, S)) are stepped in place.  Returns y
+    [B, C] (a row whose id is out of range is left as it was)."""
+    if k.dim() != 2 or v.shape != k.shape:
+        raise ValueError("k and v must both be [B, C]")
+    B, C = k.shape
+    dt = _DTYPES.get(k.dtype)
+    if dt is None or v.dtype != k.dtype:
+        raise ValueError(f"unsupported dtype {k.dtype}/{v.dtype}")
+    for name, t in (("k", k), ("v", v)):
+        _check_dev(name, t)
+    _check_dev("w", w, torch.float32)
+    _check_dev("u", u, torch.float32)
+    _check_dev("state_pool", state_pool, torch.float32)
+    _check_dev("slot_ids", slot_ids, torch.int32)
+    if state_pool.dim() != 3 or state_pool.shape[0] != 3 or state_pool.shape[2] != C:
+        raise ValueError("state_pool must be [3, S, C]")
+    if slot_ids.shape != (B,):
+        raise ValueError("slot_ids must be [B]")
+    if y is None:
+        y = torch.empty_like(k)
+    _check_dev("y", y, k.dtype)
+    rc = load().wkv4_decode_step_slots(B, C, state_pool.shape[1], _ptr(w), _ptr(u), _ptr(k), _ptr(v),
+                                       _ptr(state_pool), _ptr(slot_ids), _ptr(y), _stream(stream), dt)
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_decode_step_slots")
     return y
 
 

@@ -81,3 +81,23 @@ def test_overlapping_outputs_are_rejected():
     assert _call(si=P + 0x40000, so=P + 0x40000 + 4) == -3
     # y overlapping the state
     assert _call(si=P + 0x40000, y=P + 0x40000 + 8) == -3
+
+
+def _slots(B=2, C=16, S=5, w=P, u=P + 0x1000, k=P + 0x10000, v=P + 0x20000, pool=P + 0x40000,
+           ids=P + 0x50000, y=P + 0x30000, dtype=wkv4.F32):
+    return wkv4.load().wkv4_decode_step_slots(B, C, S, w, u, k, v, pool, ids, y, None, dtype)
+
+
+def test_slot_decode_argument_checks():
+    assert _slots(B=-1) == -1
+    assert _slots(C=-1) == -1
+    assert _slots(S=-1) == -1
+    assert _slots(dtype=5) == -2
+    assert _slots(B=0) == 0 and _slots(C=0) == 0
+    for name in ("w", "u", "k", "v", "pool", "ids", "y"):
+        assert _slots(**{name: None}) == -1, name
+    # y over the pool (3*5*16*4 = 960 bytes), the pool over k, the ids inside the pool
+    assert _slots(y=P + 0x40000 + 256) == -3
+    assert _slots(pool=P + 0x10000 + 64) == -3
+    assert _slots(ids=P + 0x40000 + 512) == -3
+    assert _slots(y=P + 0x50000 + 4) == -3

@@ -301,3 +301,70 @@ def test_golden_closed_form_fixture():
         D = np.array([[float(x) for x in r] for r in case["D_out"]])
         np.testing.assert_allclose(so[1] * np.exp(so[2]), D, rtol=1e-13)
         np.testing.assert_allclose(so[0] * np.exp(so[2]), A, rtol=1e-13, atol=1e-13 * np.max(D))
+
+
+# ---- slot-indexed decode: gather the named pool row, take the step, scatter back
+
+def test_slot_decode_matches_closed_form_on_the_named_rows():
+    rng = np.random.default_rng(77)
+    S, B, C = 5, 3, 4
+    _, _, w, u, _ = _tiny_inputs(0, C=C)
+    pool = np.stack([rng.normal(size=(S, C)), rng.uniform(0.5, 2.0, size=(S, C)),
+                     rng.uniform(-2.0, 2.0, size=(S, C))])
+    ids = np.array([4, 0, 2])
+    k = rng.normal(0.0, 2.0, size=(B, C))
+    v = rng.normal(size=(B, C))
+    y, new_pool, skipped = oracle.decode_slots(k, v, w, u, pool, ids)
+    assert skipped == 0
+    gathered = pool[:, ids, :]
+    yb, Ab, Db = brute.closed_form(k[:, None, :], v[:, None, :], w, u, gathered)
+    for b in range(B):
+        for c in range(C):
+            ref = float(yb[b][0][c])
+            assert abs(y[b, c] - ref) <= 1e-12 * max(abs(ref), abs(v[b, c])), (b, c)
+            s = ids[b]
+            e = mpmath.exp(mpmath.mpf(float(new_pool[2, s, c])))
+            D = mpmath.mpf(float(new_pool[1, s, c])) * e
+            A = mpmath.mpf(float(new_pool[0, s, c])) * e
+            assert abs(D - Db[b][c]) <= 1e-12 * Db[b][c]
+            assert abs(A - Ab[b][c]) <= 1e-12 * Db[b][c] * max(1.0, abs(v[b, c]))
+    untouched = [s for s in range(S) if s not in ids]
+    assert np.array_equal(new_pool[:, untouched, :], pool[:, untouched, :])
+
+
+def test_slot_decode_permuted_ids_follow_their_rows():
+    rng = np.random.default_rng(5)
+    S = B = 9
+    C = 4
+    _, _, w, u, _ = _tiny_inputs(1, C=C)
+    pool = np.stack([rng.normal(size=(S, C)), rng.uniform(0.5, 2.0, size=(S, C)),
+                     rng.uniform(-2.0, 2.0, size=(S, C))])
+    perm = rng.permutation(S)
+    k = rng.normal(0.0, 2.0, size=(B, C))
+    v = rng.normal(size=(B, C))
+    y, new_pool, _ = oracle.decode_slots(k, v, w, u, pool, perm)
+    # row b's result depends only on pool row perm[b] and is written back there
+    y_ref, s_ref = oracle.decode(k, v, w, u, pool[:, perm, :])
+    assert np.array_equal(y, y_ref)
+    assert np.array_equal(new_pool[:, perm, :], s_ref)
+    # the identity permutation is the plain decode
+    y_id, s_id, _ = oracle.decode_slots(k, v, w, u, pool, np.arange(S))
+    y_plain, s_plain = oracle.decode(k, v, w, u, pool)
+    assert np.array_equal(y_id, y_plain) and np.array_equal(s_id, s_plain)
+
+
+def test_slot_decode_skips_ids_outside_the_pool():
+    rng = np.random.default_rng(9)
+    S, C = 4, 4
+    _, _, w, u, _ = _tiny_inputs(2, C=C)
+    pool = np.stack([rng.normal(size=(S, C)), rng.uniform(0.5, 2.0, size=(S, C)),
+                     rng.uniform(-2.0, 2.0, size=(S, C))])
+    ids = np.array([1, -1, S, 3])
+    k = rng.normal(size=(4, C))
+    v = rng.normal(size=(4, C))
+    y, new_pool, skipped = oracle.decode_slots(k, v, w, u, pool, ids)
+    assert skipped == 2
+    assert np.all(np.isnan(y[1])) and np.all(np.isnan(y[2]))
+    assert np.all(np.isfinite(y[[0, 3]]))
+    assert np.array_equal(new_pool[:, [0, 2], :], pool[:, [0, 2], :])
+    assert not np.array_equal(new_pool[:, 1, :], pool[:, 1, :])
