@@ -24,6 +24,9 @@ L2-resident across calls by design, so the line's GB/s is effective.
 ``--workload decode_slots_b256`` is the slot-indexed decode: each call serves
 256 rows from a pool of 1024 states (wkv4_decode_step_slots), its slot ids
 drawn per call.
+``--workload token_shift_14b`` times the token shift feeding k, v and r
+(wkv4_token_shift: B=4, T=1024, C=5120, bf16, three outputs); a step is one
+call, the metric counts B*T*C elements as channel-steps.
 
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead
 (rank 0 only; other ranks exit).
@@ -398,6 +401,26 @@ def run_reference(args):
 
     wl = synth.workload(args.workload)
     config = {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C, "io_dtype": wl.dtype}
+    if wl.op == "token_shift":
+        x = synth.shift_inputs(wl)
+        for _ in range(args.warmup):
+            cpu_baseline_shift(wl, x)
+        t0 = time.perf_counter()
+        base = None
+        for _ in range(args.steps):
+            base = cpu_baseline_shift(wl, x)
+        dt = time.perf_counter() - t0
+        line = {
+            "impl": "reference", "metric": METRIC, "value": base["value"], "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     if wl.slots:
         # the oracle's slot-indexed decode over a bounded sample of the calls
         for _ in range(args.warmup):
@@ -644,6 +667,165 @@ def run_decode(args):
         dist.destroy_process_group()
 
 
+def run_shift(args):
+    """Token shift: K calls of wkv4_token_shift (CUDA graphs) over inputs that
+    rotate over more than 3x L2; device time, e2e, the oracle on the host."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from rwkv_wkv_linear_b200 import synth, wkv4
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wkv4.load()
+    wl = synth.workload(args.workload, **({"T": args.seq_len} if args.seq_len else {}))
+    x = synth.shift_inputs(wl.replace(seed=wl.seed + 1000 * rank) if rank else wl)
+    row = io_bytes(wl) // wl.T  # one [B][C] row
+    per_set = 4 * io_bytes(wl) + 2 * row  # x read, three outputs written; x_prev, x_last
+    nsets = max(2, -(-3 * L2_BYTES // per_set))
+    mk, mv, mr = (m.to(dev) for m in x["mix"])
+    xs = [x["x"].to(dev) for _ in range(nsets)]
+    xps = [x["x_prev"].to(dev) for _ in range(nsets)]
+    xls = [torch.empty_like(xps[0]) for _ in range(nsets)]
+    outs = [[torch.empty_like(xs[0]) for _ in range(3)] for _ in range(nsets)]
+    stream = torch.cuda.Stream(device=dev)
+    lib = wkv4.load()
+    dt = {"f32": wkv4.F32, "f16": wkv4.F16, "bf16": wkv4.BF16}[wl.dtype]
+    sptr = stream.cuda_stream
+
+    def call(xd, xpd, o, xld):
+        rc = lib.wkv4_token_shift(wl.B, wl.T, wl.C, xd.data_ptr(), xpd.data_ptr(), mk.data_ptr(),
+                                  mv.data_ptr(), mr.data_ptr(), o[0].data_ptr(), o[1].data_ptr(),
+                                  o[2].data_ptr(), xld.data_ptr(), sptr, dt)
+        if rc != 0:
+            raise RuntimeError(f"wkv4_token_shift failed ({rc})")
+
+    def step(i):
+        j = i % nsets
+        call(xs[j], xps[j], outs[j], xls[j])
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    K = args.steps
+    gsteps = max(1, min(args.graph_steps, K))
+    nrep, rem = divmod(K, gsteps)
+    graphs = []
+    for n in [gsteps] + ([rem] if rem else []):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                step(i)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for g in graphs:
+            g.replay()  # upload (untimed)
+    stream.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
+    clocks.start()
+    time.sleep(0.2)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(nrep):
+            graphs[0].replay()
+        if rem:
+            graphs[1].replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    ms = max_over_ranks(start.elapsed_time(end), dev)
+
+    e2e = None
+    if not args.no_e2e:
+        xh, xph = x["x"].pin_memory(), x["x_prev"].pin_memory()
+        oh = [torch.empty_like(xh).pin_memory() for _ in range(3)]
+        xlh = torch.empty_like(xph).pin_memory()
+
+        def e2e_step():
+            xs[0].copy_(xh, non_blocking=True)
+            xps[0].copy_(xph, non_blocking=True)
+            call(xs[0], xps[0], outs[0], xls[0])
+            for o_h, o_d in zip(oh, outs[0]):
+                o_h.copy_(o_d, non_blocking=True)
+            xlh.copy_(xls[0], non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, args.e2e_steps)
+        if world > 1:
+            dist.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(n_e2e):
+                e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize()
+        t2_ms = max_over_ranks(s2.elapsed_time(e2), dev)
+        e2e = {"value": job_throughput(wl.channel_steps, n_e2e, world, t2_ms), "unit": UNIT,
+               "h2d_bytes_per_step": io_bytes(wl) + row,
+               "d2h_bytes_per_step": 3 * io_bytes(wl) + row, "steps": n_e2e}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        call_bytes = 4 * io_bytes(wl) + 2 * row + 12 * wl.C
+        achieved = call_bytes / (ms / 1e3 / K) / 1e9
+        line = {
+            "metric": METRIC, "value": job_throughput(wl.channel_steps, K, world, ms),
+            "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C, "io_dtype": wl.dtype,
+                       "outputs": "xk, xv, xr and x_last", "global_batch": wl.B * world,
+                       "seq_len": wl.T, "parallelism": f"independent sequences per rank (x{world})",
+                       "l2": f"inputs rotate over {nsets} sets ({nsets * per_set / 1e6:.0f} MB > 3x L2)",
+                       "launch": f"CUDA graphs of {gsteps} calls"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "bytes_per_launch": call_bytes,
+                         "traffic": recorded_traffic(wl.name, "auto")},
+            "gpu_launches": K, "clocks": clocks.summary(), "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_shift(wl, x)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline_shift(wl, x):
+    """The oracle's token shift over the whole workload (numpy, one thread)."""
+    import oracle
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.token_shift(x["x"], x["x_prev"], x["mix"])
+        reps += 1
+        dt = time.perf_counter() - t0
+        if reps >= 3 and dt > 1.0 or dt > 20.0:
+            break
+    return {"value": wl.channel_steps * reps / dt / 1e9, "unit": UNIT, "cores": 1,
+            "kind": "oracle",
+            "sample": f"the whole workload ({wl.B}x{wl.T}x{wl.C}) x {reps} passes, fp64 numpy"}
+
+
 def _decode_as_forward(wl, rows: int = 16, calls: int = 128):
     """The first `rows` batch rows and `calls` calls of a decode workload as
     forward inputs (B = rows, T = calls), with its w, u and the zero state."""
@@ -730,6 +912,8 @@ def main():
         args.warmup = 3 if decode else 200
     if args.impl == "reference":
         run_reference(args)
+    elif synth.workload(args.workload).op == "token_shift":
+        run_shift(args)
     elif decode:
         run_decode(args)
     else:

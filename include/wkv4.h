@@ -150,6 +150,33 @@ WKV4_API int wkv4_decode_step_slots(int64_t B, int64_t C, int64_t S, const float
                                     int dtype);
 
 /*
+ * Token shift of the RWKV-4 time mix, the step before the k, v (and r)
+ * projections: each output mixes the current token's channels with the
+ * previous token's ("RWKV in a self-built engine: a second non-attention
+ * paradigm (WKV/RNN)", Reproducibility / Provenance, "Implementation":
+ * token-shift, "mix current and previous token"), read as
+ *   xk[b,t,c] = mix_k[c] x[b,t,c] + (1 - mix_k[c]) x[b,t-1,c]
+ * and likewise xv (mix_v) and xr (mix_r), with x[b,-1,c] = x_prev[b,c].
+ *   x            [B][T][C] in `dtype`.
+ *   x_prev       [B][C] in `dtype`: the token before t = 0 (the previous
+ *                call's x_last), or NULL for zeros (a sequence start).
+ *   mix_k, mix_v [C] fp32; mix_r [C] fp32 or NULL (then xr is not written).
+ *   xk, xv, xr   [B][T][C] in `dtype` (xr may be NULL when mix_r is).
+ *   x_last       [B][C] in `dtype` or NULL: receives x[:, T-1, :] (x_prev
+ *                when T == 0), the next call's x_prev.
+ * Each output is x_prev + mix (x - x_prev) in fp32, rounded once to `dtype`.
+ * Outputs must not overlap the inputs or one another (x_last included):
+ * WKV4_ERR_ALIAS.  B, T or C < 0, B > 65535 or T > 1048560: WKV4_ERR_ARG; a
+ * NULL x, mix_k, mix_v, xk, xv (or xr with mix_r given): WKV4_ERR_ARG.
+ * Chained calls with x_last fed back as x_prev equal one call over the joined
+ * T.  No allocation.
+ */
+WKV4_API int wkv4_token_shift(int64_t B, int64_t T, int64_t C, const void* x, const void* x_prev,
+                              const float* mix_k, const float* mix_v, const float* mix_r,
+                              void* xk, void* xv, void* xr, void* x_last, wkv4_stream_t stream,
+                              int dtype);
+
+/*
  * Device-side error word of the current device (bit 1: a bounded wait for a
  * TMA copy ran out; bit 2: a bounded wait for a cluster peer's partial state
  * ran out; bit 8: a slot-indexed decode row named a slot outside its pool).

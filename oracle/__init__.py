@@ -8,6 +8,7 @@ and imports nothing from it.
 * ``decode``        -- repeated T=1 forward calls with the state carried in place.
 * ``decode_slots``  -- one T=1 step per batch row on the state slot the row names
                        in a pool of states (gather, step, scatter).
+* ``token_shift``   -- the token-shift mix of the current and the previous token.
 * ``brute``         -- the closed-form sums evaluated literally in 50-digit
                        arithmetic (``oracle/brute.py``), for tiny inputs.
 
@@ -128,6 +129,28 @@ def decode_slots(k, v, w, u, pool, slot_ids):
         y[b] = yb[0]
         pool[:, s, :] = sb[:, 0, :]
     return y, pool, skipped
+
+
+def token_shift(x, x_prev, mixes):
+    """Token shift of the time mix: each output mixes the current token with
+    the previous one ("RWKV in a self-built engine: a second non-attention
+    paradigm (WKV/RNN)", Reproducibility / Provenance, "Implementation":
+    token-shift, "mix current and previous token"), read as
+        out[b, t, c] = m[c] x[b, t, c] + (1 - m[c]) x[b, t - 1, c],
+    x[b, -1, c] = x_prev[b, c] (zeros when x_prev is None), one output per mix
+    vector in ``mixes``.  x [B, T, C]; returns (list of outputs [B, T, C],
+    x_last [B, C]) in fp64.
+    """
+    x = _f64(x)
+    B, T, C = x.shape
+    prev = np.zeros((B, C)) if x_prev is None else _f64(x_prev)
+    shifted = np.concatenate([prev[:, None, :], x[:, :-1, :]], axis=1)  # x[b, t - 1]
+    outs = []
+    for m in mixes:
+        m = _f64(m)
+        outs.append(m * x + (1.0 - m) * shifted)
+    x_last = x[:, -1, :] if T > 0 else prev
+    return outs, x_last
 
 
 def empty_state(B: int, C: int) -> np.ndarray:

@@ -201,6 +201,40 @@ int wkv4_decode_step_slots(int64_t B, int64_t C, int64_t S, const float* w, cons
     return cuda_status(wkv4::launch_decode_slots(a, slot_ids, S));
 }
 
+int wkv4_token_shift(int64_t B, int64_t T, int64_t C, const void* x, const void* x_prev,
+                     const float* mix_k, const float* mix_v, const float* mix_r, void* xk,
+                     void* xv, void* xr, void* x_last, wkv4_stream_t stream, int dtype) {
+    int rc = check_common(B, T, C, dtype);
+    if (rc != WKV4_OK) return rc;
+    if (B == 0 || C == 0) return WKV4_OK;
+    const size_t es = wkv4::dtype_size(dtype);
+    const uint64_t io = (uint64_t)B * T * C * es, row = (uint64_t)B * C * es;
+    if (T == 0) {  // x_last <- x_prev (or zeros)
+        if (!x_last) return WKV4_OK;
+        if (overlap(range_of(x_last, row), range_of(x_prev, row))) return WKV4_ERR_ALIAS;
+        cudaError_t e = x_prev ? cudaMemcpyAsync(x_last, x_prev, row, cudaMemcpyDeviceToDevice,
+                                                 (cudaStream_t)stream)
+                               : cudaMemsetAsync(x_last, 0, row, (cudaStream_t)stream);
+        return cuda_status(e);
+    }
+    if (!x || !mix_k || !mix_v || !xk || !xv || (mix_r && !xr)) return WKV4_ERR_ARG;
+    if (B > 65535 || T > 65535ll * 16) return WKV4_ERR_ARG;  // grid z (rows), y (runs of 16 steps)
+    if (!mix_r) xr = nullptr;
+    const Range in[5] = {range_of(x, io), range_of(x_prev, row), range_of(mix_k, C * 4),
+                         range_of(mix_v, C * 4), range_of(mix_r, mix_r ? C * 4 : 0)};
+    const Range out[4] = {range_of(xk, io), range_of(xv, io), range_of(xr, xr ? io : 0),
+                          range_of(x_last, row)};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = 0; j < 5; ++j)
+            if (overlap(out[i], in[j])) return WKV4_ERR_ALIAS;
+        for (int j = i + 1; j < 4; ++j)
+            if (overlap(out[i], out[j])) return WKV4_ERR_ALIAS;
+    }
+    wkv4::ShiftArgs a{B, T, C, x, x_prev, {mix_k, mix_v, mix_r}, {xk, xv, xr}, x_last, dtype,
+                      (cudaStream_t)stream};
+    return cuda_status(wkv4::launch_token_shift(a));
+}
+
 int wkv4_device_error(int reset) {
     unsigned bits = 0;
     if (wkv4::read_device_error(&bits, reset != 0) != cudaSuccess) {

@@ -48,6 +48,19 @@ typedef bool (*EncodeFn)(CUtensorMap* map, const void* ptr, int dtype, int64_t B
 cudaError_t launch_scan(const FwdArgs& a, bool tma, EncodeFn encode);
 cudaError_t launch_seq(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv);
 cudaError_t launch_step(const FwdArgs& a);     // exact per-step kernel, any T >= 1
+// token shift: out[i] = mix[i] x_t + (1 - mix[i]) x_{t-1} for the non-null mix[i]
+struct ShiftArgs {
+    int64_t B, T, C;
+    const void* x;
+    const void* x_prev;
+    const float* mix[3];
+    void* out[3];
+    void* x_last;
+    int dtype;
+    cudaStream_t stream;
+};
+cudaError_t launch_token_shift(const ShiftArgs& a);  // T >= 1, B, C >= 1
+
 cudaError_t launch_decode(const FwdArgs& a);   // T == 1, vectorised when aligned
 // T == 1 over rows slots[b] of a state pool of S rows (a.state_in == a.state_out == the pool)
 cudaError_t launch_decode_slots(const FwdArgs& a, const int32_t* slots, int64_t S);

@@ -34,6 +34,7 @@ __device__ unsigned int g_device_error = 0;
 #include "wkv4_internal.h"
 #include "wkv4_scan.cuh"
 #include "wkv4_seq.cuh"
+#include "wkv4_shift.cuh"
 #include "wkv4_step.cuh"
 
 namespace wkv4 {
@@ -434,6 +435,41 @@ cudaError_t launch_decode_slots(const FwdArgs& a, const int32_t* slots, int64_t 
             case WKV4_F32: wkv4_decode_kernel<float, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
             case WKV4_F16: wkv4_decode_kernel<__half, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
             default: wkv4_decode_kernel<__nv_bfloat16, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
+        }
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_token_shift(const ShiftArgs& a) {
+    ShiftParams p{};
+    p.B = a.B;
+    p.T = a.T;
+    p.C = a.C;
+    p.x = a.x;
+    p.x_prev = a.x_prev;
+    for (int i = 0; i < 3; ++i) {
+        p.mix[i] = a.mix[i];
+        p.out[i] = a.out[i];
+    }
+    p.x_last = a.x_last;
+    const size_t es = dtype_size(a.dtype);
+    const int V = (int)(16 / es);  // 16 bytes a thread
+    bool vec = a.C % V == 0 && aligned(a.x, 16) && aligned(a.x_prev, 16) && aligned(a.x_last, 16);
+    for (int i = 0; i < 3; ++i) vec = vec && aligned(a.mix[i], 16) && aligned(a.out[i], 16);
+    const int64_t groups = (a.C + (vec ? V : 1) - 1) / (vec ? V : 1);
+    const dim3 grid((unsigned)((groups + 255) / 256), (unsigned)((a.T + kShiftRun - 1) / kShiftRun),
+                    (unsigned)a.B);
+    if (vec) {
+        switch (a.dtype) {
+            case WKV4_F32: wkv4_token_shift_kernel<float, 4><<<grid, 256, 0, a.stream>>>(p); break;
+            case WKV4_F16: wkv4_token_shift_kernel<__half, 8><<<grid, 256, 0, a.stream>>>(p); break;
+            default: wkv4_token_shift_kernel<__nv_bfloat16, 8><<<grid, 256, 0, a.stream>>>(p); break;
+        }
+    } else {
+        switch (a.dtype) {
+            case WKV4_F32: wkv4_token_shift_kernel<float, 1><<<grid, 256, 0, a.stream>>>(p); break;
+            case WKV4_F16: wkv4_token_shift_kernel<__half, 1><<<grid, 256, 0, a.stream>>>(p); break;
+            default: wkv4_token_shift_kernel<__nv_bfloat16, 1><<<grid, 256, 0, a.stream>>>(p); break;
         }
     }
     return cudaGetLastError();

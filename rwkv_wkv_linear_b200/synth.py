@@ -16,6 +16,8 @@ Workloads (sizes of the RWKV-4 models the pages discuss):
 * ``decode_slots_b256``    the same calls, each serving 256 of a pool of 1024
   conversation states (slot-indexed decode; ids drawn per call).
 * ``long_t65536``          B=1,  T=65536, C=2048, fp32 I/O, 0.1% of k set to +30.
+* ``token_shift_14b``      B=4,  T=1024,  C=5120, bf16: the token shift feeding k, v
+  and r (x, the carried token and three mix vectors).
 
 Recipe (the same for every workload; knobs per workload below):
 
@@ -62,6 +64,7 @@ class Workload:
     spike_value: float = 30.0
     steps: int = 1                 # decode workloads: number of T=1 calls
     slots: int = 0                 # slot-indexed decode: states in the pool (0: one per row)
+    op: str = "wkv"                # "wkv" or "token_shift"
 
     @property
     def channel_steps(self) -> int:
@@ -85,6 +88,8 @@ WORKLOADS = {
                             steps=1024),
     "decode_slots_b256": Workload("decode_slots_b256", B=256, T=1, C=5120, dtype="bf16", seed=3,
                                   steps=1024, slots=1024),
+    "token_shift_14b": Workload("token_shift_14b", B=4, T=1024, C=5120, dtype="bf16", seed=5,
+                                op="token_shift"),
     "long_t65536": Workload("long_t65536", B=1, T=65536, C=2048, dtype="f32", seed=4,
                             k_var=4.0, td_range=(-8.0, 2.0), u_range=(-3.0, 3.0),
                             spike_frac=0.001, spike_value=30.0),
@@ -145,6 +150,17 @@ def decode_step_inputs(wl: Workload, step: int):
     k = rng.standard_normal(shape) * math.sqrt(wl.k_var)
     v = rng.standard_normal(shape) * math.sqrt(wl.v_var)
     return _to_io(k, wl.dtype), _to_io(v, wl.dtype)
+
+
+def shift_inputs(wl: Workload) -> dict:
+    """Token-shift inputs: x [B,T,C] ~ N(0,1) and x_prev [B,C] ~ N(0,1) in the
+    I/O dtype, mix_k, mix_v, mix_r [C] ~ U(0,1) fp32 (drawn in that order from
+    default_rng(seed))."""
+    rng = np.random.default_rng(wl.seed)
+    x = rng.standard_normal((wl.B, wl.T, wl.C))
+    x_prev = rng.standard_normal((wl.B, wl.C))
+    mixes = [torch.from_numpy(rng.uniform(0.0, 1.0, size=wl.C).astype(np.float32)) for _ in range(3)]
+    return {"x": _to_io(x, wl.dtype), "x_prev": _to_io(x_prev, wl.dtype), "mix": mixes}
 
 
 def decode_slot_ids(wl: Workload, step: int) -> torch.Tensor:

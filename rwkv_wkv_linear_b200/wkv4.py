@@ -27,7 +27,7 @@ STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_DTYPE", -3: "ERR_ALIAS", -4: "ERR_CUD
 _DTYPES = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
 
 EXPORTS = ("wkv4_decode_step", "wkv4_decode_step_slots", "wkv4_device_error", "wkv4_forward",
-           "wkv4_forward_variant", "wkv4_status_string", "wkv4_version")
+           "wkv4_forward_variant", "wkv4_status_string", "wkv4_token_shift", "wkv4_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -58,6 +58,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.wkv4_decode_step.restype = i32
             lib.wkv4_decode_step_slots.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32]
             lib.wkv4_decode_step_slots.restype = i32
+            lib.wkv4_token_shift.argtypes = [i64, i64, i64] + [vp] * 10 + [i32]
+            lib.wkv4_token_shift.restype = i32
             lib.wkv4_device_error.argtypes = [i32]
             lib.wkv4_device_error.restype = i32
             lib.wkv4_status_string.argtypes = [i32]
@@ -192,6 +194,36 @@ def decode_step_slots(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torc
     if rc != 0:
         raise Wkv4Error(rc, "wkv4_decode_step_slots")
     return y
+
+
+def token_shift(x: torch.Tensor, mix_k: torch.Tensor, mix_v: torch.Tensor,
+                mix_r: Optional[torch.Tensor] = None, x_prev: Optional[torch.Tensor] = None, *,
+                x_last: Optional[torch.Tensor] = None, stream=None):
+    """wkv4_token_shift: x [B, T, C]; mixes [C] fp32; x_prev [B, C] or None.
+    Returns (xk, xv, xr or None); x_last [B, C], when given, receives x[:, -1]."""
+    if x.dim() != 3:
+        raise ValueError("x must be [B, T, C]")
+    B, T, C = x.shape
+    dt = _DTYPES.get(x.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    _check_dev("x", x)
+    for name, m in (("mix_k", mix_k), ("mix_v", mix_v), ("mix_r", mix_r)):
+        _check_dev(name, m, torch.float32)
+        if m is not None and m.shape != (C,):
+            raise ValueError(f"{name} must be [C]")
+    for name, t in (("x_prev", x_prev), ("x_last", x_last)):
+        _check_dev(name, t, x.dtype)
+        if t is not None and t.shape != (B, C):
+            raise ValueError(f"{name} must be [B, C]")
+    xk, xv = torch.empty_like(x), torch.empty_like(x)
+    xr = torch.empty_like(x) if mix_r is not None else None
+    rc = load().wkv4_token_shift(B, T, C, _ptr(x), _ptr(x_prev), _ptr(mix_k), _ptr(mix_v),
+                                 _ptr(mix_r), _ptr(xk), _ptr(xv), _ptr(xr), _ptr(x_last),
+                                 _stream(stream), dt)
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_token_shift")
+    return xk, xv, xr
 
 
 def device_error(reset: bool = True) -> int:

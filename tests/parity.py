@@ -26,12 +26,12 @@ Y_REL_16 = 1e-3
 AVG_ABS = 2e-5
 DEN_RTOL = 1e-5
 
-_MANT_BITS = {"f16": 10, "bf16": 7}
-_MIN_EXP = {"f16": -14, "bf16": -126}
+_MANT_BITS = {"f16": 10, "bf16": 7, "f32": 23}
+_MIN_EXP = {"f16": -14, "bf16": -126, "f32": -126}
 
 
 def ulp(x: np.ndarray, dtype: str) -> np.ndarray:
-    """Spacing of the fp16/bf16 grid at |x| (subnormal spacing below the normal range)."""
+    """Spacing of the fp16/bf16/fp32 grid at |x| (subnormal spacing below the normal range)."""
     m = _MANT_BITS[dtype]
     ax = np.abs(x)
     with np.errstate(divide="ignore"):

@@ -101,3 +101,24 @@ def test_slot_decode_argument_checks():
     assert _slots(pool=P + 0x10000 + 64) == -3
     assert _slots(ids=P + 0x40000 + 512) == -3
     assert _slots(y=P + 0x50000 + 4) == -3
+
+
+def _shift(B=2, T=8, C=16, x=P + 0x10000, xp=None, mk=P, mv=P + 0x1000, mr=None,
+           xk=P + 0x20000, xv=P + 0x30000, xr=None, xl=None, dtype=wkv4.F32):
+    return wkv4.load().wkv4_token_shift(B, T, C, x, xp, mk, mv, mr, xk, xv, xr, xl, None, dtype)
+
+
+def test_token_shift_argument_checks():
+    assert _shift(B=-1) == -1 and _shift(T=-1) == -1 and _shift(C=-1) == -1
+    assert _shift(dtype=3) == -2
+    assert _shift(B=0) == 0 and _shift(C=0) == 0
+    assert _shift(T=0) == 0  # no x_last: nothing to do
+    for name in ("x", "mk", "mv", "xk", "xv"):
+        assert _shift(**{name: None}) == -1, name
+    assert _shift(mr=P + 0x2000) == -1          # mix_r without xr
+    assert _shift(B=70000) == -1                # beyond the grid's batch dimension
+    # xk over x (2*8*16*4 = 1024 bytes), xv over xk, x_last over x_prev, xr over mix_r
+    assert _shift(xk=P + 0x10000 + 512) == -3
+    assert _shift(xv=P + 0x20000 + 4) == -3
+    assert _shift(xp=P + 0x40000, xl=P + 0x40000 + 8) == -3
+    assert _shift(mr=P + 0x2000, xr=P + 0x2000) == -3

@@ -368,3 +368,46 @@ def test_slot_decode_skips_ids_outside_the_pool():
     assert np.all(np.isfinite(y[[0, 3]]))
     assert np.array_equal(new_pool[:, [0, 2], :], pool[:, [0, 2], :])
     assert not np.array_equal(new_pool[:, 1, :], pool[:, 1, :])
+
+
+# ---- token shift: a per-channel mix of the current and the previous token
+
+def _shift_inputs(seed, B=3, T=9, C=5):
+    rng = np.random.default_rng(seed)
+    return rng.normal(size=(B, T, C)), rng.normal(size=(B, C))
+
+
+def test_token_shift_special_mixes_select_a_token():
+    x, xp = _shift_inputs(0)
+    ones, zeros = np.ones(5), np.zeros(5)
+    (cur, prev), last = oracle.token_shift(x, xp, [ones, zeros])
+    assert np.array_equal(cur, x)                       # mix 1: the current token
+    assert np.array_equal(prev[:, 0], xp)               # mix 0 at t = 0: the carried token
+    assert np.array_equal(prev[:, 1:], x[:, :-1])       # mix 0 later: the previous token
+    assert np.array_equal(last, x[:, -1])
+    (first,), _ = oracle.token_shift(x, None, [zeros])
+    assert np.array_equal(first[:, 0], np.zeros((3, 5)))  # a sequence start mixes with zeros
+
+
+def test_token_shift_mixes_are_per_channel():
+    x, xp = _shift_inputs(1)
+    m = np.array([1.0, 0.0, 0.5, 0.25, 1.0])
+    (out,), _ = oracle.token_shift(x, xp, [m])
+    sh = np.concatenate([xp[:, None], x[:, :-1]], axis=1)
+    assert np.array_equal(out[..., 0], x[..., 0]) and np.array_equal(out[..., 4], x[..., 4])
+    assert np.array_equal(out[..., 1], sh[..., 1])
+    assert np.allclose(out[..., 2], (x[..., 2] + sh[..., 2]) / 2, rtol=0, atol=1e-15)
+    # a convex combination: between the two tokens
+    lo, hi = np.minimum(x, sh), np.maximum(x, sh)
+    assert np.all(out >= lo - 1e-15) and np.all(out <= hi + 1e-15)
+
+
+@pytest.mark.parametrize("split", [1, 4, 8])
+def test_token_shift_chained_calls_equal_one_call(split):
+    x, xp = _shift_inputs(2)
+    m = np.random.default_rng(3).uniform(size=5)
+    (whole,), last = oracle.token_shift(x, xp, [m])
+    (a,), mid = oracle.token_shift(x[:, :split], xp, [m])
+    (b,), last2 = oracle.token_shift(x[:, split:], mid, [m])
+    assert np.array_equal(np.concatenate([a, b], axis=1), whole)
+    assert np.array_equal(last, last2)
