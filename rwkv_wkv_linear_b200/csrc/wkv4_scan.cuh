@@ -298,9 +298,16 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     };
     // Per-channel w, u and the state of a tile: a full 64-channel slice with
     // aligned pointers comes by bulk copy (lane 0 of warp 0) into a parameter
-    // slot, on that slot's barrier.
+    // slot, on that slot's barrier; any other tile (read from global memory
+    // by take_params) completes the slot's phase by a plain arrive, so that
+    // every tile takes exactly one phase of its slot and the waits' parities
+    // stay in step with the tiles.
     auto bulk_ok = [&](int64_t cc0) { return kTMA && p.bulk_params && cc0 + Cg <= C; };
     auto issue_params = [&](int slot, int bb, int64_t cc0) {
+        if (!bulk_ok(cc0)) {
+            mbar_arrive(pbar + slot);
+            return;
+        }
         float* sw = reinterpret_cast<float*>(base + lay.params(slot));
         const uint32_t nb = Cg * 4;
         const int64_t ch = (int64_t)bb * C + cc0;
@@ -331,7 +338,7 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
             }
             mbar_init(mbar + warp, 1);
             fence_mbar_init();
-            if (warp == 0 && bulk_ok(c0)) issue_params(0, b, c0);
+            if (warp == 0) issue_params(0, b, c0);
             issue_rows(0, b, c0);
         }
         __syncwarp();
@@ -604,7 +611,7 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
             if (kTMA && more) {
                 __syncwarp();  // every lane has read the rows
                 if (lane == 0) {
-                    if (warp == 0 && bulk_ok(nc0)) issue_params((j + 1) & 1, nb, nc0);
+                    if (warp == 0) issue_params((j + 1) & 1, nb, nc0);
                     issue_k(0, nb, nc0);
                 }
             }

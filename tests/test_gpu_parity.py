@@ -212,3 +212,15 @@ def test_forward_under_cuda_graph(cuda_device):
     graph.replay()
     torch.cuda.synchronize()
     check(x, "f16", y.cpu(), s.cpu(), "graph")
+
+
+@pytest.mark.parametrize("shape", [(128, 100, 2048, "f16"), (48, 600, 1000, "bf16"), (40, 300, 512, "f32")],
+                         ids=lambda s: "B%dT%dC%d_%s" % s)
+def test_persistent_clusters_walk_many_tiles(cuda_device, shape):
+    """Far more channel tiles than clusters that fit at once (one round per
+    tile): every cluster walks many tiles, alternating its parameter and
+    aggregate slots, with the carried state and partial last tiles."""
+    B, T, C, dt = shape
+    x = synth.custom(B, T, C, dt, seed=B + T + C, random_state=True, k_var=2.0)
+    y, s = gpu_forward(x, cuda_device, wkv4.KERNEL_SCAN)
+    check(x, dt, y, s, f"persistent {shape}")
