@@ -160,13 +160,24 @@ def algorithmic_bytes(wl):
     return 3 * io_bytes(wl) + (state if wl.random_state else 0) + state + 8 * wl.C
 
 
-def kernel_source_hash():
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without its comments and blank lines (string and
+    character literals kept), so that the hash below changes with the code only."""
+    import re
+    token = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'', re.S)
+    out = token.sub(lambda m: "" if m.group(0)[0] == "/" else m.group(0), text)
+    return "\n".join(line.rstrip() for line in out.splitlines() if line.strip())
+
+
+def kernel_source_hash(csrc=None):
+    """Hash of the kernel sources' code (comments and blank lines left out):
+    a recorded DRAM-traffic figure applies only while it matches."""
     import hashlib
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "rwkv_wkv_linear_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "rwkv_wkv_linear_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -3,37 +3,40 @@
 //
 // A cluster of NC CTAs owns one channel tile (Cg = 64 channels of one batch
 // row, one channel pair per lane) and walks T in rounds of NC segments of
-// Ts = NW L steps; CTA rank r takes segment round * NC + r.  NW (warps per
-// CTA) and NC are chosen at launch so that, where the GPU can hold it, the
-// whole T is one round of one wave.  Inside a CTA each warp owns one chunk of
-// L steps; its rows arrive by their own TMA box and mbarrier, so a warp
-// starts as soon as its rows land.  Per round:
+// Ts = NW L steps; CTA rank r takes segment round * NC + r.  Inside a CTA
+// each warp owns one chunk of L steps; its rows arrive by their own TMA box
+// and mbarrier, so a warp starts as soon as its rows land.  Per round:
 //   1. every warp summarises its chunk from the empty state (chunk_phase1
 //      with stash: the per-step numerators and denominators of its outputs
 //      go to tensor memory);
-//   2. once every summary is in, warp 0 joins them (a balanced tree) into the
-//      segment's aggregate and pushes it into the shared memory of every CTA
-//      of the cluster by asynchronous DSMEM stores that complete on the
-//      receiving CTA's barrier of that round's slot; the state contribution
-//      before each chunk: one round, every warp joins the summaries before
-//      its own; several rounds, warp 0 scans them in place (one chain, which
-//      also gives the aggregate);
-//   3. once all NC aggregates of the round have landed, warp 1 folds them,
-//      from the state carried into the round, into the state at the segment
-//      start (into shared memory) and the state carried into the next round;
+//   2. once every summary is in, warp 0 joins them into the segment's
+//      aggregate and pushes it into the shared memory of every CTA of the
+//      cluster by asynchronous DSMEM stores that complete on the receiving
+//      CTA's barrier of that exchange's slot;
+//   3. once all NC aggregates have landed, warp 1 folds them, from the state
+//      carried into the round, into the state at the segment start (into
+//      shared memory) and the state carried into the next round;
 //   4. after a CTA barrier every warp joins the segment start state with its
-//      chunk's prefix and computes its chunk's outputs from the stash.
-// Only warps 0 and 1 run the scan and the fold: every warp running them
-// would queue on the transcendental and conversion pipe they lean on.
-// One round: y is staged in the warp's k rows and sent out by one TMA store.
+//      chunk's prefix (the summaries of the chunks before it) and computes its
+//      chunk's outputs from the stash.
+// Only warps 0, 1 (and 2) run the scan, the fold (and the chunk prefixes):
+// every warp running them would queue on the transcendental and conversion
+// pipe they lean on.
+// One round (kMulti false): persistent clusters, as many as the GPU holds at
+// once, walk the channel tiles tile, tile + G, ...; warp 0 joins the
+// summaries as a balanced tree, warp 2 scans the chunk prefixes into their
+// own array; a warp's k rows (and warp 0's parameters) of the next tile load
+// right after its summary pass, y is staged in its v rows and sent out by one
+// TMA store, and the next tile's v rows follow once the store has read them.
 // Several rounds (kMulti) are software-pipelined: a warp's rows take the next
 // round's load right after its summary pass; round r + 1's steps 1 and 2 run
-// before round r's step 4, and warp 1 folds round r + 1 after its step 4 of
+// before round r's step 4 (warp 0 scans the summaries in place, one chain that
+// also gives the aggregate), and warp 1 folds round r + 1 after its step 4 of
 // round r, so the aggregates travel while the warps work.  The chunk
-// summaries, the stash, the segment start state and the aggregates alternate
-// between two slots; y goes straight from registers to global memory.  There
-// is no global scratch: all exchange is through cluster shared memory.  Every
-// wait is bounded.
+// summaries, the stash and the segment start state alternate between two
+// slots; y goes straight from registers to global memory.  Aggregates always
+// alternate between two slots.  There is no global scratch: all exchange is
+// through cluster shared memory.  Every wait is bounded.
 #pragma once
 
 #include <cooperative_groups.h>
