@@ -8,11 +8,14 @@
 // Methods table "Precision"; Reproducibility / Provenance "Implementation").
 //
 // Kernels (one translation unit, so they share the device error word):
-//   wkv4_scan_kernel    (wkv4_scan.cuh) chunked scan, tiles chained through
-//                       a thread-block cluster; TMA in, TMA out.
+//   wkv4_scan_kernel    (wkv4_scan.cuh) chunked scan, time segments chained
+//                       through a thread-block cluster; TMA in, TMA out (one
+//                       round) or stores from registers (several rounds).
 //   wkv4_seq_kernel     (wkv4_seq.cuh) channel-parallel, sequential over T.
-//   wkv4_step_kernel, wkv4_decode_kernel, wkv4_copy_state_kernel
-//                       (wkv4_step.cuh) per-step paths.
+//   wkv4_step_kernel, wkv4_decode_kernel (plain or slot-indexed),
+//   wkv4_copy_state_kernel  (wkv4_step.cuh) per-step paths.
+//   wkv4_token_shift_kernel (wkv4_shift.cuh) the token shift before the
+//                       k, v, r projections.
 // No tensor cores: nothing here is a dense contraction; the work is bound by
 // HBM bandwidth (k, v read once, y written once).
 #include <cuda.h>
