@@ -122,3 +122,28 @@ def test_token_shift_argument_checks():
     assert _shift(xv=P + 0x20000 + 4) == -3
     assert _shift(xp=P + 0x40000, xl=P + 0x40000 + 8) == -3
     assert _shift(mr=P + 0x2000, xr=P + 0x2000) == -3
+
+
+def test_binding_rejects_host_tensors_and_bad_shapes():
+    """The Python binding checks devices, dtypes and shapes before any CUDA
+    call (host tensors, so no GPU is needed to reach these errors)."""
+    import torch
+    k = torch.zeros(2, 8, 16)
+    w = torch.zeros(16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        wkv4.forward(k, k, w, w)
+    with pytest.raises(ValueError, match="\\[B, T, C\\]"):
+        wkv4.forward(k[0], k[0], w, w)
+    with pytest.raises(ValueError, match="unsupported dtype"):
+        wkv4.forward(k.double(), k.double(), w, w)
+    with pytest.raises(ValueError, match="\\[B, C\\]"):
+        wkv4.decode_step(k, k, w, w, torch.zeros(3, 2, 16))
+    with pytest.raises(ValueError, match="\\[B, C\\]"):
+        wkv4.decode_step_slots(k, k, w, w, torch.zeros(3, 4, 16), torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        wkv4.decode_step_slots(k[:, 0], k[:, 0], w, w, torch.zeros(3, 4, 16),
+                               torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="\\[B, T, C\\]"):
+        wkv4.token_shift(k[0], w, w)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        wkv4.token_shift(k, w, w)
