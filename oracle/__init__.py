@@ -9,6 +9,9 @@ and imports nothing from it.
 * ``decode_slots``  -- one T=1 step per batch row on the state slot the row names
                        in a pool of states (gather, step, scatter).
 * ``token_shift``   -- the token-shift mix of the current and the previous token.
+* ``forward_gated`` / ``decode_gated`` -- the receptance gate of the time mix,
+                       y = sigmoid(r) * wkv, applied to ``forward`` / ``decode``.
+* ``combine_states`` -- one segment's state followed by another's (T split).
 * ``brute``         -- the closed-form sums evaluated literally in 50-digit
                        arithmetic (``oracle/brute.py``), for tiny inputs.
 
@@ -151,6 +154,52 @@ def token_shift(x, x_prev, mixes):
         outs.append(m * x + (1.0 - m) * shifted)
     x_last = x[:, -1, :] if T > 0 else prev
     return outs, x_last
+
+
+def sigmoid(r):
+    """The logistic function 1 / (1 + e^{-r}) in fp64, elementwise (0 for r
+    below about -709, where e^{-r} overflows, and 1 above about 37)."""
+    r = _f64(r)
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-r))
+
+
+def forward_gated(k, v, r, w, u, state_in=None, *, nthreads: int = 1):
+    """The WKV forward with the receptance gate of the time mix applied to its
+    output: y = sigmoid(r) * wkv elementwise, r [B, T, C] ("RWKV in a
+    self-built engine: a second non-attention paradigm (WKV/RNN)", abstract
+    and Reproducibility / Provenance, "Implementation": time-mix gating;
+    "RWKV-4 14B", "Every architecture field": the time mix's receptance
+    matrix).  The pages name the gate and the receptance but not the gate's
+    function; it is read as the logistic sigmoid.  The state does not depend
+    on r.  Returns (y [B, T, C], state_out [3, B, C]) in fp64.
+    """
+    y, s = forward(k, v, w, u, state_in, nthreads=nthreads)
+    return y * sigmoid(r), s
+
+
+def decode_gated(k, v, r, w, u, state):
+    """One T=1 step over k, v, r [B, C] with the receptance gate on its output:
+    returns (sigmoid(r) * wkv [B, C], new state [3, B, C])."""
+    y, s = decode(k, v, w, u, state)
+    return y * sigmoid(r), s
+
+
+def combine_states(x, y, n, w):
+    """State x followed by a segment of n steps whose state from the empty
+    state is y (both [3, B, C] planes num, den, max in natural units; n an
+    int; w [C]): the state after both, X's numerator and denominator decayed
+    by e^{n w}:  A = e^{n w} A_x + A_y,  D = e^{n w} D_x + D_y,  returned as a
+    (num, den, max) triple with the max-trick (max = max(p_x + n w, p_y)).
+    The state carried across a split of T ("An RNN that claims to match
+    transformers, now in chatbot form", "The interesting bit": the state is
+    the whole history).  fp64.
+    """
+    x, y, w = _f64(x), _f64(y), _f64(w)
+    px = x[2] + n * w
+    p = np.maximum(px, y[2])
+    ex, ey = np.exp(px - p), np.exp(y[2] - p)
+    return np.stack([ex * x[0] + ey * y[0], ex * x[1] + ey * y[1], p])
 
 
 def empty_state(B: int, C: int) -> np.ndarray:
