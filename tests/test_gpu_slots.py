@@ -50,9 +50,12 @@ def test_slot_decode_matches_oracle_over_steps(cuda_device, dt, C):
                                    u.to(cuda_device), pool_dev, ids.to(cuda_device))
         torch.cuda.synchronize()
         state_before = pool_ref[:, ids.numpy(), :]
+        abs_pool = pool_ref.copy()
+        abs_pool[0] = np.abs(abs_pool[0])
+        ya, _, _ = oracle.decode_slots(k, v.abs(), w, u, abs_pool, ids)
         y_ref, pool_ref, skipped = oracle.decode_slots(k, v, w, u, pool_ref, ids)
         assert skipped == 0
-        parity.check_y(y.cpu(), y_ref, v, dt, f"slots {dt} C={C} y step {step}")
+        parity.check_y(y.cpu(), y_ref, v, dt, f"slots {dt} C={C} y step {step}", y_abs=ya)
         got = pool_dev.cpu().double().numpy()
         idx = ids.numpy()
         parity.check_state(got[:, idx, :], pool_ref[:, idx, :], v, state_before,

@@ -18,7 +18,8 @@ def test_gate_accepts_the_oracle_rounded_to_io_dtype():
         x = synth.forward_inputs(wl)
         y, s = oracle.forward(x["k"], x["v"], x["w"], x["u"], x["state_in"])
         y_io = torch.from_numpy(y).to(wl.torch_dtype)
-        parity.check_y(y_io, y, x["v"], dt)
+        ya = parity.y_abs(x["k"], x["v"], x["w"], x["u"], x["state_in"])
+        parity.check_y(y_io, y, x["v"], dt, y_abs=ya)
         parity.check_state(s.astype(np.float32), s, x["v"], x["state_in"])
 
 
@@ -67,3 +68,35 @@ def test_ulp_grid():
     assert parity.ulp(np.array([3.0]), "f16")[0] == 2.0 ** -9
     assert parity.ulp(np.array([0.0]), "f16")[0] == 2.0 ** -24
     assert parity.ulp(np.array([1e-6]), "f16")[0] == 2.0 ** -24
+
+
+def test_y_abs_bounds_the_output_and_equals_it_for_positive_terms():
+    x = synth.forward_inputs(synth.workload("rwkv4_169m_prefill", B=2, T=64, C=32))
+    y, _ = oracle.forward(x["k"], x["v"], x["w"], x["u"], x["state_in"])
+    ya = parity.y_abs(x["k"], x["v"], x["w"], x["u"], x["state_in"])
+    assert np.all(ya >= np.abs(y) * (1 - 1e-12))
+    s = x["state_in"].clone()
+    s[0] = s[0].abs()
+    yp, _ = oracle.forward(x["k"], x["v"].abs(), x["w"], x["u"], s)
+    np.testing.assert_array_equal(parity.y_abs(x["k"], x["v"].abs(), x["w"], x["u"], s), yp)
+
+
+def test_16_bit_gate_rejects_outputs_that_lose_bits_near_zero():
+    """An fp16 output whose fp32 computation lost its low half (a 2^-12
+    relative error against the terms) fails where the terms cancel, while
+    the exact output rounded once to fp16 passes."""
+    wl = synth.workload("rwkv4_169m_prefill", B=2, T=256, C=64)
+    x = synth.forward_inputs(wl)
+    y, _ = oracle.forward(x["k"], x["v"], x["w"], x["u"], x["state_in"])
+    ya = parity.y_abs(x["k"], x["v"], x["w"], x["u"], x["state_in"])
+    parity.check_y(torch.from_numpy(y).half(), y, x["v"], "f16", y_abs=ya)
+    rng = np.random.default_rng(0)
+    noisy = y + rng.choice([-1.0, 1.0], size=y.shape) * 2.0 ** -12 * ya
+    with pytest.raises(AssertionError):
+        parity.check_y(torch.from_numpy(noisy).half(), y, x["v"], "f16", y_abs=ya)
+
+
+def test_16_bit_gate_needs_y_abs():
+    y = np.zeros((1, 2, 2))
+    with pytest.raises(ValueError):
+        parity.check_y(y, y, y, "bf16")
