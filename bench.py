@@ -5,12 +5,15 @@
 
 A step is one wkv4_forward call (the whole hot path: load, chunk summaries,
 segment chaining, outputs, final state) over one batch of the workload,
-default ``rwkv4_169m_prefill`` (B=8, T=1024, C=768, fp16 k/v/y, random fp32
-state in and out).  Inputs are seeded synthetic data (rwkv_wkv_linear_b200.synth)
-resident in HBM; the timed steps rotate over enough input sets that their
-total exceeds 3x the L2 cache, so no step reads another step's data from L2.
-The K steps run as CUDA-graph replays of the public call; the device time of
-the region (CUDA events on the launching stream) is max-reduced over ranks.
+default ``long_t65536`` (B=1, T=65536, C=2048, fp32 k/v/y, 0.1% of k spiked to
++30, fp32 state out: the largest single-GPU workload, 1.6 GB a call).  Inputs
+are seeded synthetic data (rwkv_wkv_linear_b200.synth) resident in HBM; the
+timed steps rotate over enough input sets that their total exceeds 3x the L2
+cache, so no step reads another step's data from L2.  The K steps run as
+CUDA-graph replays of the public call, right after about 0.25 s of untimed
+replays (so the timed region starts on a busy GPU, not one waking from idle);
+the device time of the region (CUDA events on the launching stream) is
+max-reduced over ranks.
 
 Under torchrun each rank processes its own batch (independent sequences, no
 collective on the data path): weak scaling.
@@ -61,7 +64,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=None,
                     help="untimed steps (default 200 calls; 3 loops for a decode workload)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="rwkv4_169m_prefill")
+    ap.add_argument("--workload", default="long_t65536")
     ap.add_argument("--variant", default="auto", choices=sorted(VARIANTS))
     ap.add_argument("--graph-steps", type=int, default=500,
                     help="forward calls captured per CUDA graph")
@@ -85,27 +88,64 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """SM clock and throttle reasons sampled while the GPU works: NVML every
+    few milliseconds from a thread of this process (reads only), else
+    nvidia-smi every 50 ms.  summary(t0, t1) keeps the samples taken between
+    host times t0 and t1 (the timed region), or, when the region is shorter
+    than the sampling period, the last samples before t1."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.rows = []
+    def __init__(self, gpu: str, period_s: float = 0.002):
+        self.gpu = gpu
+        self.period = period_s
+        self.rows = []  # (host time, sm MHz, max MHz, set of reasons)
         self.proc = None
         self.t = None
+        self.stop_flag = threading.Event()
+        self.source = None
 
     def start(self):
         try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.gpu.encode()) if self.gpu.startswith("GPU-")
+                 else pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu)))
+            bits = {"hw_slowdown": pynvml.nvmlClocksThrottleReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksThrottleReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksThrottleReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksThrottleReasonSwPowerCap}
+            mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                        r = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                        self.rows.append((time.perf_counter(), sm, mx,
+                                          {n for n, b in bits.items() if r & b}))
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+
+            self.t = threading.Thread(target=poll, daemon=True)
+            self.t.start()
+            self.source = f"nvml every {self.period * 1e3:.0f} ms"
+            return
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
+        self.source = "nvidia-smi every 50 ms"
         self.t = threading.Thread(target=self._read, daemon=True)
         self.t.start()
 
@@ -113,9 +153,15 @@ class ClockSampler:
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) >= 9:
-                self.rows.append(parts)
+                try:
+                    reasons = {n for n, val in zip(self.NAMES, parts[5:9])
+                               if val.lower().startswith("active")}
+                    self.rows.append((time.perf_counter(), float(parts[1]), float(parts[2]), reasons))
+                except ValueError:
+                    pass
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -125,22 +171,23 @@ class ClockSampler:
         if self.t is not None:
             self.t.join(timeout=5)
 
-    def summary(self):
-        sm = []
-        mx = None
+    def summary(self, t0=None, t1=None):
+        rows = list(self.rows)
+        window = "timed region"
+        if t0 is not None and t1 is not None:
+            inside = [r for r in rows if t0 <= r[0] <= t1]
+            if len(inside) < 3:
+                inside = [r for r in rows if r[0] <= t1][-5:]
+                window = "last samples up to the end of the timed region (region shorter than the period)"
+            rows = inside
+        sm = [r[1] for r in rows]
         reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in self.rows:
-            try:
-                sm.append(float(r[1]))
-                mx = float(r[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, r[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        for r in rows:
+            reasons |= r[3]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": rows[-1][2] if rows else None,
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source,
+                "window": window}
 
 
 def dist_env():
@@ -210,10 +257,70 @@ def cpu_baseline(wl, x):
         dt = time.perf_counter() - t0
         if reps >= 3 and dt > 1.0 or dt > 20.0:
             break
-    return {"value": wl.channel_steps * reps / dt / 1e9, "unit": UNIT, "cores": cores,
-            "kind": "oracle",
+    value = wl.channel_steps * reps / dt / 1e9
+    # one core, on the first channels of the workload (about 2 s of work)
+    BC = wl.B * wl.C
+    n_ch = max(1, min(BC, int(2.0 * value * 1e9 / max(1, cores) / wl.T)))
+    smp = _ref_sample(x, wl, n_ch)
+    t0 = time.perf_counter()
+    oracle.forward(*smp, nthreads=1)
+    value_1core = n_ch * wl.T / (time.perf_counter() - t0) / 1e9
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"the whole workload ({wl.B}x{wl.T}x{wl.C}) x {reps} passes, fp64 C "
-                      f"recurrence, {cores} threads over channels"}
+                      f"recurrence, {cores} threads over channels",
+            "value_1core": value_1core,
+            "sample_1core": f"{n_ch} of {BC} channels x all {wl.T} steps, one thread"}
+
+
+def start_clocks(dev, local):
+    import torch
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
+    clocks.start()
+    return clocks
+
+
+def busy_warmup(stream, graph, seconds: float = 0.25):
+    """Untimed replays for about `seconds`, ending right before the timed
+    region: its first steps then run at the clocks of a busy GPU."""
+    import torch
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        while time.perf_counter() - t0 < seconds:
+            graph.replay()
+            stream.synchronize()
+
+
+def host_call_us(wl, ks, vs, w, u, sis, ys, sos, variant, stream, calls: int = 200) -> float:
+    """Host time of one wkv4_forward_variant call through the C ABI with its
+    arguments already marshalled (argument checks, launch shape, tensor maps,
+    launch): the cost an eager caller pays per call on top of the kernel."""
+    import ctypes
+
+    import torch
+    from rwkv_wkv_linear_b200 import wkv4
+    lib = wkv4.load()
+    dt = {"f32": wkv4.F32, "f16": wkv4.F16, "bf16": wkv4.BF16}[wl.dtype]
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    args = [(wl.B, wl.T, wl.C, w.data_ptr(), u.data_ptr(), ks[j].data_ptr(), vs[j].data_ptr(),
+             sis[j].data_ptr() if sis[j] is not None else None, ys[j].data_ptr(),
+             sos[j].data_ptr(), sp, dt, variant) for j in range(len(ks))]
+    for a in args:  # first calls of each set (tensor maps encoded once)
+        lib.wkv4_forward_variant(*a)
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(3):
+        t0 = time.perf_counter()
+        for i in range(calls):
+            rc = lib.wkv4_forward_variant(*args[i % len(args)])
+        t1 = time.perf_counter()
+        torch.cuda.synchronize()
+        if rc != 0:
+            raise RuntimeError(f"wkv4_forward_variant failed ({rc})")
+        us = (t1 - t0) / calls * 1e6
+        best = us if best is None else min(best, us)
+    return best
 
 
 def max_over_ranks(ms: float, device=None) -> float:
@@ -293,15 +400,13 @@ def run_native(args):
             rem_graph.replay()
     stream.synchronize()
 
-    props = torch.cuda.get_device_properties(dev)
-    uuid = getattr(props, "uuid", None)
-    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
-    clocks.start()
-    time.sleep(0.2)
+    clocks = start_clocks(dev, local)
+    busy_warmup(stream, main_graph)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    t_region0 = time.perf_counter()
     start.record(stream)
     with torch.cuda.stream(stream):
         for _ in range(nrep):
@@ -310,12 +415,14 @@ def run_native(args):
             rem_graph.replay()
     end.record(stream)
     torch.cuda.synchronize()
+    t_region1 = time.perf_counter()
     if world > 1:
         dist.barrier()
     clocks.stop()
     ms = max_over_ranks(start.elapsed_time(end), dev)
     if wkv4.device_error() != 0:
         raise RuntimeError("device-side wait ran out during the timed region")
+    host_us = host_call_us(wl, ks, vs, w, u, sis, ys, sos, variant, stream)
 
     # end to end through the C ABI from pinned host buffers
     e2e = None
@@ -340,7 +447,10 @@ def run_native(args):
             for _ in range(3):
                 e2e_step()
         torch.cuda.synchronize()
-        n_e2e = max(1, args.e2e_steps)
+        h2d = 2 * io_bytes(wl) + (12 * wl.B * wl.C if sih is not None else 0)
+        d2h = io_bytes(wl) + 12 * wl.B * wl.C
+        # about 4 GB of copies at most (three steps at the least)
+        n_e2e = max(3, min(args.e2e_steps, int(4e9 // (h2d + d2h))))
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -352,8 +462,6 @@ def run_native(args):
         e2.record(stream)
         torch.cuda.synchronize()
         t2_ms = max_over_ranks(s2.elapsed_time(e2), dev)
-        h2d = 2 * io_bytes(wl) + (12 * wl.B * wl.C if sih is not None else 0)
-        d2h = io_bytes(wl) + 12 * wl.B * wl.C
         e2e = {"value": job_throughput(wl.channel_steps, n_e2e, world, t2_ms),
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": n_e2e}
@@ -383,14 +491,17 @@ def run_native(args):
                        "l2": f"inputs rotate over {nsets} sets ({nsets * per_set / 1e6:.0f} MB "
                              f"> 3x L2)",
                        "launch": f"CUDA graphs of {gsteps} calls, {nrep}+{1 if rem else 0} "
-                                 "replays (one untimed upload replay each)"},
+                                 "replays (one untimed upload replay each)",
+                       "untimed": f"{args.warmup} warm-up calls before capture; about 0.25 s of "
+                                  "replays right before the timed region"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
                          "bytes_per_launch": algorithmic_bytes(wl),
                          "traffic": recorded_traffic(wl.name, args.variant)},
             "gpu_launches": K,
-            "clocks": clocks.summary(),
+            "clocks": clocks.summary(t_region0, t_region1),
             "e2e": e2e,
+            "host_us_per_call": host_us,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, x)
@@ -568,21 +679,20 @@ def run_decode(args):
     stream.synchronize()
 
     K = args.steps
-    props = torch.cuda.get_device_properties(dev)
-    uuid = getattr(props, "uuid", None)
-    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
-    clocks.start()
-    time.sleep(0.2)
+    clocks = start_clocks(dev, local)
+    busy_warmup(stream, g)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    t_region0 = time.perf_counter()
     start.record(stream)
     with torch.cuda.stream(stream):
         for _ in range(K):
             g.replay()
     end.record(stream)
     torch.cuda.synchronize()
+    t_region1 = time.perf_counter()
     if world > 1:
         dist.barrier()
     clocks.stop()
@@ -667,7 +777,7 @@ def run_decode(args):
                          "bytes_per_launch": call_bytes, "effective": True,
                          "traffic": recorded_traffic(wl.name, "auto")},
             "gpu_launches": calls,
-            "clocks": clocks.summary(),
+            "clocks": clocks.summary(t_region0, t_region1),
             "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -739,15 +849,13 @@ def run_shift(args):
         for g in graphs:
             g.replay()  # upload (untimed)
     stream.synchronize()
-    props = torch.cuda.get_device_properties(dev)
-    uuid = getattr(props, "uuid", None)
-    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
-    clocks.start()
-    time.sleep(0.2)
+    clocks = start_clocks(dev, local)
+    busy_warmup(stream, graphs[0])
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    t_region0 = time.perf_counter()
     start.record(stream)
     with torch.cuda.stream(stream):
         for _ in range(nrep):
@@ -756,6 +864,7 @@ def run_shift(args):
             graphs[1].replay()
     end.record(stream)
     torch.cuda.synchronize()
+    t_region1 = time.perf_counter()
     if world > 1:
         dist.barrier()
     clocks.stop()
@@ -812,7 +921,7 @@ def run_shift(args):
                          "frac": achieved / peak, "peak_kind": peak_kind,
                          "bytes_per_launch": call_bytes,
                          "traffic": recorded_traffic(wl.name, "auto")},
-            "gpu_launches": K, "clocks": clocks.summary(), "e2e": e2e,
+            "gpu_launches": K, "clocks": clocks.summary(t_region0, t_region1), "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_shift(wl, x)

@@ -33,6 +33,10 @@ Recipe (the same for every workload; knobs per workload below):
 * Decode draws w, u from ``default_rng(seed)`` and each call's k, v from
   ``default_rng([seed, step])``; a slot-indexed decode call's ids are the first
   B of a permutation of the pool drawn from ``default_rng([seed, step, 1])``.
+* The receptance r of the gated forward (y = sigmoid(r) wkv) is drawn from a
+  stream of its own, ``default_rng([seed, 7])`` (a decode call's from
+  ``default_rng([seed, step, 2])``), as N(0, 4) rounded to the I/O dtype, so
+  that k, v and the state are the same draws with or without it.
 """
 
 from __future__ import annotations
@@ -135,6 +139,18 @@ def forward_inputs(wl: Workload) -> dict:
         k.reshape(-1)[idx] = wl.spike_value
     return {"w": w, "u": u, "k": _to_io(k, wl.dtype), "v": _to_io(v, wl.dtype),
             "state_in": state}
+
+
+def receptance(wl: Workload, var: float = 4.0) -> torch.Tensor:
+    """r [B, T, C] ~ N(0, var) in the I/O dtype for the gated forward."""
+    rng = np.random.default_rng([wl.seed, 7])
+    return _to_io(rng.standard_normal((wl.B, wl.T, wl.C)) * math.sqrt(var), wl.dtype)
+
+
+def decode_receptance(wl: Workload, step: int, var: float = 4.0) -> torch.Tensor:
+    """r [B, C] of gated decode call number ``step``."""
+    rng = np.random.default_rng([wl.seed, step, 2])
+    return _to_io(rng.standard_normal((wl.B, wl.C)) * math.sqrt(var), wl.dtype)
 
 
 def decode_params(wl: Workload):
