@@ -201,10 +201,11 @@ def io_bytes(wl):
 
 
 def algorithmic_bytes(wl):
-    """k, v read + y written (I/O dtype) + state in (when given) and out (fp32
-    triples) + w, u (fp32)."""
+    """k, v (and r, gated) read + y written (I/O dtype) + state in (when given)
+    and out (fp32 triples) + w, u (fp32)."""
     state = 12 * wl.B * wl.C
-    return 3 * io_bytes(wl) + (state if wl.random_state else 0) + state + 8 * wl.C
+    return ((4 if wl.gated else 3) * io_bytes(wl) + (state if wl.random_state else 0) + state
+            + 8 * wl.C)
 
 
 def _code_only(text: str) -> str:
@@ -250,9 +251,16 @@ def cpu_baseline(wl, x):
     import oracle
     cores = len(os.sched_getaffinity(0))
     oracle.forward(x["k"][:1, :8], x["v"][:1, :8], x["w"], x["u"], None, nthreads=cores)
+    r = None
+    if wl.gated:
+        from rwkv_wkv_linear_b200 import synth
+        r = synth.receptance(wl)
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.forward(x["k"], x["v"], x["w"], x["u"], x["state_in"], nthreads=cores)
+        if r is None:
+            oracle.forward(x["k"], x["v"], x["w"], x["u"], x["state_in"], nthreads=cores)
+        else:
+            oracle.forward_gated(x["k"], x["v"], r, x["w"], x["u"], x["state_in"], nthreads=cores)
         reps += 1
         dt = time.perf_counter() - t0
         if reps >= 3 and dt > 1.0 or dt > 20.0:
@@ -292,7 +300,8 @@ def busy_warmup(stream, graph, seconds: float = 0.25):
             stream.synchronize()
 
 
-def host_call_us(wl, ks, vs, w, u, sis, ys, sos, variant, stream, calls: int = 200) -> float:
+def host_call_us(wl, ks, vs, w, u, sis, ys, sos, variant, stream, rs=None,
+                 calls: int = 200) -> float:
     """Host time of one wkv4_forward_variant call through the C ABI with its
     arguments already marshalled (argument checks, launch shape, tensor maps,
     launch): the cost an eager caller pays per call on top of the kernel."""
@@ -303,17 +312,20 @@ def host_call_us(wl, ks, vs, w, u, sis, ys, sos, variant, stream, calls: int = 2
     lib = wkv4.load()
     dt = {"f32": wkv4.F32, "f16": wkv4.F16, "bf16": wkv4.BF16}[wl.dtype]
     sp = ctypes.c_void_p(stream.cuda_stream)
-    args = [(wl.B, wl.T, wl.C, w.data_ptr(), u.data_ptr(), ks[j].data_ptr(), vs[j].data_ptr(),
-             sis[j].data_ptr() if sis[j] is not None else None, ys[j].data_ptr(),
-             sos[j].data_ptr(), sp, dt, variant) for j in range(len(ks))]
+    gated = rs is not None and rs[0] is not None
+    fn = lib.wkv4_forward_gated_variant if gated else lib.wkv4_forward_variant
+    args = [(wl.B, wl.T, wl.C, w.data_ptr(), u.data_ptr(), ks[j].data_ptr(), vs[j].data_ptr())
+            + ((rs[j].data_ptr(),) if gated else ())
+            + (sis[j].data_ptr() if sis[j] is not None else None, ys[j].data_ptr(),
+               sos[j].data_ptr(), sp, dt, variant) for j in range(len(ks))]
     for a in args:  # first calls of each set (tensor maps encoded once)
-        lib.wkv4_forward_variant(*a)
+        fn(*a)
     torch.cuda.synchronize()
     best = None
     for _ in range(3):
         t0 = time.perf_counter()
         for i in range(calls):
-            rc = lib.wkv4_forward_variant(*args[i % len(args)])
+            rc = fn(*args[i % len(args)])
         t1 = time.perf_counter()
         torch.cuda.synchronize()
         if rc != 0:
@@ -359,11 +371,12 @@ def run_native(args):
     wl = synth.workload(args.workload, **({"T": args.seq_len} if args.seq_len else {}))
     x = synth.forward_inputs(wl.replace(seed=wl.seed + 1000 * rank) if rank else wl)
 
-    per_set = 2 * io_bytes(wl) + io_bytes(wl) + 24 * wl.B * wl.C
+    per_set = (3 if wl.gated else 2) * io_bytes(wl) + io_bytes(wl) + 24 * wl.B * wl.C
     nsets = max(2, -(-3 * L2_BYTES // per_set))
     nsets = min(nsets, max(2, int(20e9 // per_set)))
     w, u = x["w"].to(dev), x["u"].to(dev)
     ks = [x["k"].to(dev) for _ in range(nsets)]
+    rs = [synth.receptance(wl).to(dev) for _ in range(nsets)] if wl.gated else [None] * nsets
     vs = [x["v"].to(dev) for _ in range(nsets)]
     sis = [x["state_in"].to(dev) if x["state_in"] is not None else None for _ in range(nsets)]
     ys = [torch.empty_like(ks[0]) for _ in range(nsets)]
@@ -372,8 +385,12 @@ def run_native(args):
 
     def step(i):
         j = i % nsets
-        wkv4.forward(ks[j], vs[j], w, u, sis[j], y=ys[j], state_out=sos[j], variant=variant,
-                     stream=stream)
+        if wl.gated:
+            wkv4.forward_gated(ks[j], vs[j], rs[j], w, u, sis[j], y=ys[j], state_out=sos[j],
+                               variant=variant, stream=stream)
+        else:
+            wkv4.forward(ks[j], vs[j], w, u, sis[j], y=ys[j], state_out=sos[j], variant=variant,
+                         stream=stream)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -422,7 +439,7 @@ def run_native(args):
     ms = max_over_ranks(start.elapsed_time(end), dev)
     if wkv4.device_error() != 0:
         raise RuntimeError("device-side wait ran out during the timed region")
-    host_us = host_call_us(wl, ks, vs, w, u, sis, ys, sos, variant, stream)
+    host_us = host_call_us(wl, ks, vs, w, u, sis, ys, sos, variant, stream, rs)
 
     # end to end through the C ABI from pinned host buffers
     e2e = None
@@ -433,13 +450,21 @@ def run_native(args):
         soh = torch.empty((3, wl.B, wl.C), dtype=torch.float32).pin_memory()
         kd, vd, yd, sod = ks[0], vs[0], ys[0], sos[0]
         sid = sis[0]
+        rh = synth.receptance(wl).pin_memory() if wl.gated else None
+        rd = rs[0]
 
         def e2e_step():
             kd.copy_(kh, non_blocking=True)
             vd.copy_(vh, non_blocking=True)
             if sih is not None:
                 sid.copy_(sih, non_blocking=True)
-            wkv4.forward(kd, vd, w, u, sid, y=yd, state_out=sod, variant=variant, stream=stream)
+            if wl.gated:
+                rd.copy_(rh, non_blocking=True)
+                wkv4.forward_gated(kd, vd, rd, w, u, sid, y=yd, state_out=sod, variant=variant,
+                                   stream=stream)
+            else:
+                wkv4.forward(kd, vd, w, u, sid, y=yd, state_out=sod, variant=variant,
+                             stream=stream)
             yh.copy_(yd, non_blocking=True)
             soh.copy_(sod, non_blocking=True)
 
@@ -447,7 +472,7 @@ def run_native(args):
             for _ in range(3):
                 e2e_step()
         torch.cuda.synchronize()
-        h2d = 2 * io_bytes(wl) + (12 * wl.B * wl.C if sih is not None else 0)
+        h2d = (3 if wl.gated else 2) * io_bytes(wl) + (12 * wl.B * wl.C if sih is not None else 0)
         d2h = io_bytes(wl) + 12 * wl.B * wl.C
         # about 4 GB of copies at most (three steps at the least)
         n_e2e = max(3, min(args.e2e_steps, int(4e9 // (h2d + d2h))))
@@ -485,6 +510,7 @@ def run_native(args):
             "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
                        "io_dtype": wl.dtype, "state_in": "random" if wl.random_state else "none",
+                       "gate": "y = sigmoid(r) wkv, r ~ N(0, 4)" if wl.gated else "none",
                        "global_batch": wl.B * world, "seq_len": wl.T,
                        "parallelism": f"independent sequences per rank (x{world})",
                        "kernel": args.variant,

@@ -110,6 +110,35 @@ WKV4_API int wkv4_forward_variant(int64_t B, int64_t T, int64_t C, const float* 
                          float* state_out, wkv4_stream_t stream, int dtype, int variant);
 
 /*
+ * The forward with the receptance gate of the time mix applied to its output:
+ *   y = sigmoid(r) * wkv  elementwise,  sigmoid(r) = 1 / (1 + e^{-r}),
+ * the gating that follows the WKV recurrence in the time mix ("RWKV in a
+ * self-built engine: a second non-attention paradigm (WKV/RNN)", abstract
+ * and Reproducibility / Provenance, "Implementation": time-mix gating;
+ * "RWKV-4 14B", "Every architecture field": the time mix's receptance
+ * matrix).  The pages name the gate but not its function; the logistic
+ * sigmoid is the reading taken.  Fused into the output pass: one more
+ * exponential a channel-step, no extra pass over y.
+ *   r          [B][T][C] in `dtype` (the receptance), required when B, T and
+ *              C are all non-zero (else WKV4_ERR_ARG).  y must not overlap r,
+ *              nor may state_out (WKV4_ERR_ALIAS).
+ * Every other argument, the state, the return codes and the alignment rules
+ * (r takes part in them like k and v) are those of wkv4_forward; the state
+ * does not depend on r.  No allocation.
+ */
+WKV4_API int wkv4_forward_gated(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                                const void* k, const void* v, const void* r,
+                                const float* state_in, void* y, float* state_out,
+                                wkv4_stream_t stream, int dtype);
+
+/* wkv4_forward_gated with an explicit kernel choice (as wkv4_forward_variant). */
+WKV4_API int wkv4_forward_gated_variant(int64_t B, int64_t T, int64_t C, const float* w,
+                                        const float* u, const void* k, const void* v,
+                                        const void* r, const float* state_in, void* y,
+                                        float* state_out, wkv4_stream_t stream, int dtype,
+                                        int variant);
+
+/*
  * One decode step (T = 1) for B sequences, updating the state in place.
  *   w, u     [C] fp32.
  *   k, v     [B][C] in `dtype`.
@@ -120,6 +149,16 @@ WKV4_API int wkv4_forward_variant(int64_t B, int64_t T, int64_t C, const float* 
  */
 WKV4_API int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float* u, const void* k,
                      const void* v, float* state, void* y, wkv4_stream_t stream, int dtype);
+
+/*
+ * wkv4_decode_step with the receptance gate on its output: y = sigmoid(r) *
+ * wkv (see wkv4_forward_gated).  r [B][C] in `dtype`, required; y must not
+ * overlap it.  Equal, bit for bit, to wkv4_forward_gated with T = 1 and
+ * state_in == state_out.
+ */
+WKV4_API int wkv4_decode_step_gated(int64_t B, int64_t C, const float* w, const float* u,
+                                    const void* k, const void* v, const void* r, float* state,
+                                    void* y, wkv4_stream_t stream, int dtype);
 
 /*
  * One decode step (T = 1) for B sequences whose states live in a pool of S
@@ -175,6 +214,28 @@ WKV4_API int wkv4_token_shift(int64_t B, int64_t T, int64_t C, const void* x, co
                               const float* mix_k, const float* mix_v, const float* mix_r,
                               void* xk, void* xv, void* xr, void* x_last, wkv4_stream_t stream,
                               int dtype);
+
+/*
+ * The state after two consecutive segments of one sequence, from the state
+ * after the first and the second's own state: x (the state after the first
+ * segment, or NULL for the empty state) followed by y (the state of a
+ * segment of n_steps steps from the empty state), per channel
+ *   A = e^{n_steps w} A_x + A_y,   D = e^{n_steps w} D_x + D_y,
+ * returned as a (num, den, max) triple with the max-trick.  The state is the
+ * sequence's whole history ("An RNN that claims to match transformers, now
+ * in chatbot form", "The interesting bit"), so a sequence split over T --
+ * across devices, each summarising its own segment from the empty state --
+ * is joined by this combine: the state entering segment r is the combine of
+ * the segments before it, in order.
+ *   w          [C] fp32 decay (as for wkv4_forward).
+ *   x, y, out  [3][B][C] fp32 (planes num, den, max).  out may be x or y
+ *              itself; any other overlap (or out over w) is WKV4_ERR_ALIAS.
+ * B, C or n_steps < 0, a NULL w, y or out: WKV4_ERR_ARG.  Asynchronous on
+ * `stream`, no allocation.
+ */
+WKV4_API int wkv4_state_combine(int64_t B, int64_t C, const float* w, int64_t n_steps,
+                                const float* x, const float* y, float* out,
+                                wkv4_stream_t stream);
 
 /*
  * Device-side error word of the current device (bit 1: a bounded wait for a

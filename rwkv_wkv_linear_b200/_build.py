@@ -14,6 +14,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libwkv4.so")
+# the bounds-checked build (WKV4_CHECKED: every global index checked, fault
+# injection switches read from the environment), for the failure tests
+CHECKED_LIB = os.path.join(PKG, "libwkv4_checked.so")
 SOURCES = [os.path.join(CSRC, "wkv4_kernels.cu"), os.path.join(CSRC, "wkv4_api.cpp")]
 
 
@@ -45,6 +48,20 @@ def stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps())
 
 
+def stale_at(path: str) -> bool:
+    if not os.path.exists(path):
+        return True
+    t = os.path.getmtime(path)
+    return any(os.path.getmtime(d) > t for d in deps())
+
+
+def build_checked(force: bool = False, verbose: bool = False) -> str:
+    """Compile libwkv4_checked.so (WKV4_CHECKED) when stale."""
+    if not force and not stale_at(CHECKED_LIB):
+        return CHECKED_LIB
+    return build(force=True, verbose=verbose, out=CHECKED_LIB, defines=("WKV4_CHECKED",))
+
+
 def build(force: bool = False, verbose: bool = False, out: str = LIB, defines=()) -> str:
     """Compile libwkv4.so (or `out`, with extra -D `defines`) when stale."""
     if out == LIB and not defines and not force and not stale():
@@ -60,3 +77,4 @@ def build(force: bool = False, verbose: bool = False, out: str = LIB, defines=()
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))
+    print(build_checked(force="--force" in sys.argv, verbose=True))

@@ -52,8 +52,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 3-D map over a [B][T][C] tensor (dims innermost first: C, T, B) with a
 // box of box_c channels x box_t steps x 1 batch row; out-of-range elements
 // read as zero and are skipped on store.
-bool encode_btc(CUtensorMap* map, const void* ptr, int dtype, int64_t B, int64_t T, int64_t C,
-                int box_c, int box_t) {
+bool encode_btc_uncached(CUtensorMap* map, const void* ptr, int dtype, int64_t B, int64_t T,
+                         int64_t C, int box_c, int box_t) {
     auto fn = encode_fn();
     if (!fn) return false;
     const size_t es = wkv4::dtype_size(dtype);
@@ -69,11 +69,51 @@ bool encode_btc(CUtensorMap* map, const void* ptr, int dtype, int64_t B, int64_t
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// encode_btc_uncached through a small per-thread cache: a map depends only on
+// its arguments, and callers run the same buffers call after call (encoding
+// one costs about a microsecond of host time, three a call).
+struct MapKey {
+    const void* ptr;
+    int64_t B, T, C;
+    int dtype, box_c, box_t;
+    bool operator==(const MapKey& o) const {
+        return ptr == o.ptr && B == o.B && T == o.T && C == o.C && dtype == o.dtype &&
+               box_c == o.box_c && box_t == o.box_t;
+    }
+};
+
+bool encode_btc(CUtensorMap* map, const void* ptr, int dtype, int64_t B, int64_t T, int64_t C,
+                int box_c, int box_t) {
+    constexpr int kEntries = 64;
+    struct Entry {
+        MapKey key;
+        CUtensorMap map;
+        bool used;
+    };
+    static thread_local Entry cache[kEntries];
+    static thread_local int next = 0;
+    const MapKey key{ptr, B, T, C, dtype, box_c, box_t};
+    for (int i = 0; i < kEntries; ++i) {
+        if (cache[i].used && cache[i].key == key) {
+            *map = cache[i].map;
+            return true;
+        }
+    }
+    if (!encode_btc_uncached(map, ptr, dtype, B, T, C, box_c, box_t)) return false;
+    Entry& e = cache[next];
+    next = (next + 1) % kEntries;
+    e.key = key;
+    e.map = *map;
+    e.used = true;
+    return true;
+}
+
 // TMA needs 16-byte aligned bases and row strides that are multiples of 16 bytes.
 bool tma_eligible(const FwdArgs& a) {
     const size_t es = wkv4::dtype_size(a.dtype);
     return (a.C * (int64_t)es) % 16 == 0 && is_aligned(a.k, 16) && is_aligned(a.v, 16) &&
-           is_aligned(a.y, 16) && a.T < (1ll << 31) && a.C < (1ll << 31) && a.B < (1ll << 31);
+           is_aligned(a.y, 16) && is_aligned(a.r, 16) && a.T < (1ll << 31) &&
+           a.C < (1ll << 31) && a.B < (1ll << 31);
 }
 
 int check_common(int64_t B, int64_t T, int64_t C, int dtype) {
@@ -87,12 +127,14 @@ int check_alias(const FwdArgs& a) {
     const uint64_t io = (uint64_t)a.B * a.T * a.C * es;
     const uint64_t st = (uint64_t)3 * a.B * a.C * 4;
     const Range ry = range_of(a.y, io), rk = range_of(a.k, io), rv = range_of(a.v, io);
+    const Range rr = range_of(a.r, io);
     const Range rw = range_of(a.w, a.C * 4), ru = range_of(a.u, a.C * 4);
     const Range rsi = range_of(a.state_in, st), rso = range_of(a.state_out, st);
     if (overlap(ry, rk) || overlap(ry, rv) || overlap(ry, rw) || overlap(ry, ru) ||
-        overlap(ry, rsi) || overlap(ry, rso))
+        overlap(ry, rsi) || overlap(ry, rso) || overlap(ry, rr))
         return WKV4_ERR_ALIAS;
-    if (overlap(rso, rk) || overlap(rso, rv) || overlap(rso, rw) || overlap(rso, ru))
+    if (overlap(rso, rk) || overlap(rso, rv) || overlap(rso, rw) || overlap(rso, ru) ||
+        overlap(rso, rr))
         return WKV4_ERR_ALIAS;
     if (overlap(rso, rsi) && a.state_in != a.state_out) return WKV4_ERR_ALIAS;
     return WKV4_OK;
@@ -111,11 +153,12 @@ int run_scan(const FwdArgs& a, bool want_tma) {
 int run_seq(const FwdArgs& a) {
     if (!tma_eligible(a) || !is_aligned(a.y, 16)) return run_scan(a, false);
     const wkv4::Geom g = wkv4::seq_geom(a.dtype);
-    CUtensorMap tk, tv;
+    CUtensorMap tk, tv, tr;
     if (!encode_btc(&tk, a.k, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t) ||
-        !encode_btc(&tv, a.v, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t))
+        !encode_btc(&tv, a.v, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t) ||
+        (a.r && !encode_btc(&tr, a.r, a.dtype, a.B, a.T, a.C, g.box_c, g.box_t)))
         return WKV4_ERR_CUDA;
-    return cuda_status(wkv4::launch_seq(a, &tk, &tv));
+    return cuda_status(wkv4::launch_seq(a, &tk, &tv, a.r ? &tr : &tk));
 }
 
 // Kernel choice of wkv4_forward.  The sequential kernel needs enough channel
@@ -167,6 +210,22 @@ int wkv4_forward_variant(int64_t B, int64_t T, int64_t C, const float* w, const 
     return forward_impl(a, variant);
 }
 
+int wkv4_forward_gated(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                       const void* k, const void* v, const void* r, const float* state_in,
+                       void* y, float* state_out, wkv4_stream_t stream, int dtype) {
+    return wkv4_forward_gated_variant(B, T, C, w, u, k, v, r, state_in, y, state_out, stream,
+                                      dtype, WKV4_KERNEL_AUTO);
+}
+
+int wkv4_forward_gated_variant(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                               const void* k, const void* v, const void* r,
+                               const float* state_in, void* y, float* state_out,
+                               wkv4_stream_t stream, int dtype, int variant) {
+    if (T > 0 && B > 0 && C > 0 && !r) return WKV4_ERR_ARG;
+    FwdArgs a{B, T, C, w, u, k, v, state_in, y, state_out, dtype, (cudaStream_t)stream, r};
+    return forward_impl(a, variant);
+}
+
 int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float* u, const void* k,
                      const void* v, float* state, void* y, wkv4_stream_t stream, int dtype) {
     int rc = check_common(B, 1, C, dtype);
@@ -174,6 +233,19 @@ int wkv4_decode_step(int64_t B, int64_t C, const float* w, const float* u, const
     if (B == 0 || C == 0) return WKV4_OK;
     if (!w || !u || !k || !v || !y || !state) return WKV4_ERR_ARG;
     FwdArgs a{B, 1, C, w, u, k, v, state, y, state, dtype, (cudaStream_t)stream};
+    rc = check_alias(a);
+    if (rc != WKV4_OK) return rc;
+    return cuda_status(wkv4::launch_decode(a));
+}
+
+int wkv4_decode_step_gated(int64_t B, int64_t C, const float* w, const float* u, const void* k,
+                           const void* v, const void* r, float* state, void* y,
+                           wkv4_stream_t stream, int dtype) {
+    int rc = check_common(B, 1, C, dtype);
+    if (rc != WKV4_OK) return rc;
+    if (B == 0 || C == 0) return WKV4_OK;
+    if (!w || !u || !k || !v || !r || !y || !state) return WKV4_ERR_ARG;
+    FwdArgs a{B, 1, C, w, u, k, v, state, y, state, dtype, (cudaStream_t)stream, r};
     rc = check_alias(a);
     if (rc != WKV4_OK) return rc;
     return cuda_status(wkv4::launch_decode(a));
@@ -233,6 +305,20 @@ int wkv4_token_shift(int64_t B, int64_t T, int64_t C, const void* x, const void*
     wkv4::ShiftArgs a{B, T, C, x, x_prev, {mix_k, mix_v, mix_r}, {xk, xv, xr}, x_last, dtype,
                       (cudaStream_t)stream};
     return cuda_status(wkv4::launch_token_shift(a));
+}
+
+int wkv4_state_combine(int64_t B, int64_t C, const float* w, int64_t n_steps, const float* x,
+                       const float* y, float* out, wkv4_stream_t stream) {
+    if (B < 0 || C < 0 || n_steps < 0) return WKV4_ERR_ARG;
+    if (B == 0 || C == 0) return WKV4_OK;
+    if (!w || !y || !out) return WKV4_ERR_ARG;
+    if (B * C > (int64_t)UINT32_MAX * 256) return WKV4_ERR_ARG;
+    const uint64_t st = (uint64_t)3 * B * C * 4;
+    const Range ro = range_of(out, st), rx = range_of(x, st), ry = range_of(y, st);
+    if (overlap(ro, range_of(w, C * 4))) return WKV4_ERR_ALIAS;
+    if (overlap(ro, rx) && out != x) return WKV4_ERR_ALIAS;
+    if (overlap(ro, ry) && out != y) return WKV4_ERR_ALIAS;
+    return cuda_status(wkv4::launch_state_combine(B, C, w, n_steps, x, y, out, (cudaStream_t)stream));
 }
 
 int wkv4_device_error(int reset) {

@@ -50,6 +50,44 @@ __device__ __forceinline__ float rcp_approx(float x) {
 __device__ __forceinline__ f2 ex2_2(f2 x) { return pk(ex2(lo(x)), ex2(hi(x))); }
 __device__ __forceinline__ f2 rcp2(f2 x) { return pk(rcp_approx(lo(x)), rcp_approx(hi(x))); }
 
+// ------------------------------------------------------ receptance gate
+//
+// The time mix's output is gated by the receptance: y = sigmoid(r) wkv
+// ("RWKV in a self-built engine: a second non-attention paradigm
+// (WKV/RNN)", abstract and Reproducibility / Provenance, "Implementation":
+// time-mix gating; "RWKV-4 14B", "Every architecture field": the time mix's
+// receptance matrix), with sigmoid(r) = 1 / (1 + e^{-r}).  On the outputs'
+// fast paths it is folded into the one reciprocal they already take:
+//   y = num / (den (1 + e^{-r})),  den (1 + g) = fma(den, g, den),  g = e^{-r},
+// one more exponential and one FMA a channel-step.  e^{-r} overflows to
+// +inf below r = -88, where the quotient is 0: the gate's limit.
+
+// g = e^{-r} for a channel pair
+__device__ __forceinline__ f2 gate_g2(f2 r) { return ex2_2(mul2(r, pk(-kLog2e, -kLog2e))); }
+
+// sigmoid(r) y for one channel (the per-step paths)
+__device__ __forceinline__ float gate_one(float y, float r) {
+    return y * rcp_approx(1.f + ex2(-r * kLog2e));
+}
+
+// No gate: the outputs' paths compile without it.
+struct NoGate {
+    static constexpr bool kOn = false;
+    __device__ __forceinline__ f2 operator()(int) const { return 0ull; }
+};
+
+// A gate of the outputs' fast paths: f(i) gives g = e^{-r} of step i's pair.
+template <typename F>
+struct FnGate {
+    static constexpr bool kOn = true;
+    F f;
+    __device__ __forceinline__ f2 operator()(int i) const { return f(i); }
+};
+template <typename F>
+__device__ __forceinline__ FnGate<F> fn_gate(F f) {
+    return FnGate<F>{f};
+}
+
 // ------------------------------------------------------- pair I/O by dtype
 
 template <typename IO> struct Pair;
@@ -341,10 +379,13 @@ __device__ __noinline__ void chunk_phase3_general(const PairRef& r, const IO* sk
     }
 }
 
-template <typename IO, int L, typename OutPair, typename OutOne>
+// With a gate (Gate::kOn), gate(i) gives g = e^{-r_i} of step i's pair and
+// the fast loop divides by den (1 + g); the general path's out_one applies
+// the gate itself.
+template <typename IO, int L, typename OutPair, typename OutOne, typename Gate = NoGate>
 __device__ __forceinline__ void chunk_phase3(const PairRef& r, const IO* sk, const IO* sv, int stride,
                                              int col, int n, const St (&S)[2], const PairConsts& cc,
-                                             OutPair out_pair, OutOne out_one) {
+                                             OutPair out_pair, OutOne out_one, Gate gate = Gate()) {
     if (n <= 0) return;
     bool f3[2];
     float a0[2], b0[2];
@@ -365,7 +406,9 @@ __device__ __forceinline__ void chunk_phase3(const PairRef& r, const IO* sk, con
             const f2 e = ex2_2(fma2(Pair<IO>::load(sk + i * stride + col), l2e, nref));
             const f2 ev = mul2(e, Pair<IO>::load(sv + i * stride + col));
             // (A + e^u e v) / (D + e^u e), then A <- e^w A + e v, D <- e^w D + e
-            const f2 y = mul2(fma2(cc.eu, ev, Ah), rcp2(fma2(cc.eu, e, Dh)));
+            f2 den = fma2(cc.eu, e, Dh);
+            if constexpr (Gate::kOn) den = fma2(den, gate(i), den);
+            const f2 y = mul2(fma2(cc.eu, ev, Ah), rcp2(den));
             Ah = fma2(cc.ew, Ah, ev);
             Dh = fma2(cc.ew, Dh, e);
             out_pair(i, y);
@@ -414,12 +457,14 @@ __device__ __noinline__ void chunk_exact_global(const IO* gk, const IO* gv, int6
 // path from k, v in global memory (gk, gv: the pair's first channel at the
 // chunk's first step, row stride `stride`; ok[j]: channel j exists) through
 // out_one(i, j, y).
-template <typename IO, int L, typename OutPair, typename OutOne>
+// With a gate (Gate::kOn), gate(i) gives g = e^{-r_i} of step i's pair and
+// y_i = num / (den (1 + g)); the exact path's out_one applies the gate itself.
+template <typename IO, int L, typename OutPair, typename OutOne, typename Gate = NoGate>
 __device__ __forceinline__ void chunk_phase3_stash(const PairRef& r, int n, const St (&S)[2],
                                                    const PairConsts& cc, uint32_t taddr,
                                                    const IO* gk, const IO* gv, int64_t stride,
                                                    bool ok0, bool ok1, OutPair out_pair,
-                                                   OutOne out_one) {
+                                                   OutOne out_one, Gate gate = Gate()) {
     static_assert(L % 4 == 0, "stash: whole column groups");
     if (n <= 0) return;
     bool f3[2];
@@ -441,7 +486,9 @@ __device__ __forceinline__ void chunk_phase3_stash(const PairRef& r, int n, cons
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
                     const f2 N = pku(st[4 * s], st[4 * s + 1]), Dn = pku(st[4 * s + 2], st[4 * s + 3]);
-                    out_pair(4 * q + s, mul2(fma2(f, al, N), rcp2(fma2(f, be, Dn))));
+                    f2 den = fma2(f, be, Dn);
+                    if constexpr (Gate::kOn) den = fma2(den, gate(4 * q + s), den);
+                    out_pair(4 * q + s, mul2(fma2(f, al, N), rcp2(den)));
                     f = mul2(f, cc.ew);
                 }
             }
@@ -455,7 +502,9 @@ __device__ __forceinline__ void chunk_phase3_stash(const PairRef& r, int n, cons
                     if (4 * q + s < n) {
                         const f2 N = pku(st[4 * s], st[4 * s + 1]);
                         const f2 Dn = pku(st[4 * s + 2], st[4 * s + 3]);
-                        out_pair(4 * q + s, mul2(fma2(f, al, N), rcp2(fma2(f, be, Dn))));
+                        f2 den = fma2(f, be, Dn);
+                        if constexpr (Gate::kOn) den = fma2(den, gate(4 * q + s), den);
+                        out_pair(4 * q + s, mul2(fma2(f, al, N), rcp2(den)));
                         f = mul2(f, cc.ew);
                     }
                 }

@@ -33,6 +33,24 @@
 
 namespace wkv4 {
 
+// The device error word (per device; wkv4_device_error reads and clears it):
+// the bits of wkv4_internal.h, set by the kernels with atomicOr.
+__device__ unsigned int g_device_error = 0;
+
+// Checked builds (WKV4_CHECKED): every global index is checked against the
+// extent of its buffer before the access; one outside it sets kErrBounds in
+// the error word and the access is skipped.  Other builds compile the check
+// to `true`.
+#ifdef WKV4_CHECKED
+__device__ __forceinline__ bool in_range(int64_t i, int64_t n) {
+    if (i >= 0 && i < n) return true;
+    atomicOr(&g_device_error, kErrBounds);
+    return false;
+}
+#else
+__device__ __forceinline__ constexpr bool in_range(int64_t, int64_t) { return true; }
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr double kLog2eD = 1.4426950408889634;
 constexpr double kLn2D = 0.6931471805599453;
@@ -112,14 +130,19 @@ __device__ __forceinline__ void exact_update(St& s, float k, float v, double w2)
 // per-step kernel, where one step's rounding is carried to the next call.
 // Of the two scale factors of each half step the one at the max is exactly
 // 1 (exp2f(0)), so only the other one is evaluated: the same bits as taking
-// both, with half the exponentials.
-__device__ __forceinline__ float step_nat(St& s, float k, float v, float w, float u) {
+// both, with half the exponentials.  kGate: the output gated by the
+// receptance r, sigmoid(r) y = num / (den (1 + e^{-r})) (e^{-r} = inf below
+// r = -88 gives 0, the gate's limit).
+template <bool kGate = false>
+__device__ __forceinline__ float step_nat(St& s, float k, float v, float w, float u, float r = 0.f) {
     const double kd = k;
     // output: q = max(p, u + k)
     const double d1 = s.p - ((double)u + kd);
     const float f = exp2f((float)-fabs(d1) * kLog2e);
     const float f1 = d1 >= 0.0 ? 1.f : f, f2 = d1 >= 0.0 ? f : 1.f;
-    const float y = __fdividef(fmaf(f1, s.a, f2 * v), fmaf(f1, s.b, f2));
+    float den = fmaf(f1, s.b, f2);
+    if constexpr (kGate) den = fmaf(den, exp2f(-r * kLog2e), den);
+    const float y = __fdividef(fmaf(f1, s.a, f2 * v), den);
     // state: q2 = max(p + w, k)
     const double pw = s.p + (double)w;
     const double d2 = pw - kd;
@@ -137,7 +160,10 @@ __device__ __forceinline__ bool fast_ok(float kmax, float kmin, float u, float w
 
 // fp32 state buffers <-> kernel state.  On the way out the max is rounded to
 // fp32 and the rounding error d (natural units, |d| <= half an ulp of the
-// max) is folded into a and b as a(1 + d), b(1 + d) -- e^d to first order.
+// max) is folded into a and b as a e^d = a + a (e^d - 1), b likewise, with
+// e^d - 1 from expm1f (d itself to within its last bit while |d| is below
+// about 2^-12; a max of 10^5 nats, after a long decay with nothing new, has
+// |d| up to 2^-5, where the first-order d alone would be off by d^2 / 2).
 __device__ __forceinline__ St load_state_log2(const float* __restrict__ s, int64_t BC, int64_t ch) {
     return {s[ch], s[BC + ch], (double)s[2 * BC + ch] * kLog2eD};
 }
@@ -145,7 +171,7 @@ __device__ __forceinline__ St load_state_log2(const float* __restrict__ s, int64
 __device__ __forceinline__ void store_state_nat_d(float* __restrict__ s, int64_t BC, int64_t ch,
                                                   float a, float b, double p_nat) {
     const float pf = (float)p_nat;
-    const float d = (float)(p_nat - (double)pf);
+    const float d = expm1f((float)(p_nat - (double)pf));
     s[ch] = fmaf(a, d, a);
     s[BC + ch] = fmaf(b, d, b);
     s[2 * BC + ch] = pf;
@@ -265,11 +291,12 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase (about kWaitRounds x 1 ms at most);
-// false when it ran out.
+// Bounded wait on an mbarrier phase (about `rounds` x 1 ms at most); false
+// when it ran out.
 constexpr uint32_t kWaitRounds = 1000;
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitRounds; ++i)
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint32_t rounds = kWaitRounds) {
+    for (uint32_t i = 0; i < rounds; ++i)
         if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     return false;
 }
@@ -291,6 +318,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Prefetch of a box of a tiled tensor into L2 (no shared-memory destination,
+// nothing to wait for).
+__device__ __forceinline__ void tma_prefetch_3d_l2(const CUtensorMap* map, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y,
@@ -353,8 +389,9 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitRounds; ++i)
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity,
+                                                          uint32_t rounds = kWaitRounds) {
+    for (uint32_t i = 0; i < rounds; ++i)
         if (mbar_try_wait_cluster(bar, parity, 1000000u)) return true;
     return false;
 }

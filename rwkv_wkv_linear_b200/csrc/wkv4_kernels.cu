@@ -26,14 +26,10 @@
 #include <climits>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/wkv4.h"
 #include "wkv4_device.cuh"
-
-namespace wkv4 {
-__device__ unsigned int g_device_error = 0;
-}
-
 #include "wkv4_internal.h"
 #include "wkv4_scan.cuh"
 #include "wkv4_seq.cuh"
@@ -86,21 +82,120 @@ static int env_int(const char* name, int dflt) {
 
 constexpr size_t kMaxSmem = 227 * 1024;
 constexpr int kTmemColumns = 512;  // tensor-memory columns per SM
+constexpr int kMaxDevices = 64;
 
-// Dynamic shared memory to request for a scan CTA: its layout's bytes, raised
-// where needed so that no more CTAs fit on an SM than the SM's tensor memory
-// serves (a CTA allocates `cols` columns at its start and holds them to its
-// end; an allocation that cannot be met would wait for another CTA's release).
-static size_t scan_smem_request(size_t bytes, int cols) {
-    int dev = 0, per_sm = 233472, reserved = 1024;
-    if (cudaGetDevice(&dev) == cudaSuccess) {
-        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+// Per-device limits the launch shapes are worked out from, queried once per
+// device (the launchers run on every call; attribute queries are not free).
+struct DeviceAttrs {
+    int smem_per_sm = 233472, smem_reserved = 1024, reg_file = 65536, max_threads = 2048,
+        max_blocks = 32;
+};
+
+static const DeviceAttrs& device_attrs() {
+    static DeviceAttrs attrs[kMaxDevices];
+    static std::once_flag once[kMaxDevices];
+    static DeviceAttrs fallback;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return fallback;
     }
-    const int cap = kTmemColumns / cols;  // CTAs per SM the tensor memory serves
-    // (cap + 1) CTAs of (request + reserved) bytes each do not fit on an SM
-    const size_t floor_bytes = (size_t)per_sm / (size_t)(cap + 1) + 1;
-    size_t need = floor_bytes > (size_t)reserved ? floor_bytes - (size_t)reserved : 0;
+    std::call_once(once[dev], [dev] {
+        DeviceAttrs& a = attrs[dev];
+        cudaDeviceGetAttribute(&a.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&a.smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+        cudaDeviceGetAttribute(&a.reg_file, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&a.max_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+        cudaDeviceGetAttribute(&a.max_blocks, cudaDevAttrMaxBlocksPerMultiprocessor, dev);
+        cudaGetLastError();
+    });
+    return attrs[dev];
+}
+
+// Tuning overrides of the scan's launch shape, read from the environment
+// once per process: WKV4_SCAN_NW (warps per CTA), WKV4_SCAN_CLUSTER (cluster
+// size), WKV4_SCAN_WAVES=1 (one cluster per channel tile with one round).
+struct ScanOverrides {
+    int nw, nc, waves;
+};
+
+// Limit of each bounded device-side wait, in rounds of about 1 ms.  Checked
+// builds (WKV4_CHECKED) take WKV4_WAIT_ROUNDS from the environment, so that a
+// test can make a wait run out quickly.
+static uint32_t wait_rounds() {
+#ifdef WKV4_CHECKED
+    static const int r = env_int("WKV4_WAIT_ROUNDS", 0);
+    if (r > 0) return (uint32_t)r;
+#endif
+    return kWaitRounds;
+}
+
+// Fault injection, in checked builds only (WKV4_CHECKED), read once from
+// WKV4_FAULT:
+//   launch:N   the N-th kernel launch of the process (1-based) is made with an
+//              empty grid, which the runtime rejects (cudaErrorInvalid-
+//              Configuration) without running anything: the launch error path
+//              of every entry point, with no GPU fault;
+//   exchange   no scan CTA pushes its segment aggregate, so every CTA's
+//              bounded wait for its peers' aggregates runs out (with a short
+//              limit from WKV4_WAIT_ROUNDS): the expiry path of the exchange.
+// Production builds compile none of it.
+struct FaultPlan {
+    long launch_at = 0;  // 0: none
+    bool exchange = false;
+};
+
+static const FaultPlan& fault_plan() {
+    static const FaultPlan plan = [] {
+        FaultPlan f;
+#ifdef WKV4_CHECKED
+        if (const char* e = std::getenv("WKV4_FAULT")) {
+            if (std::strncmp(e, "launch:", 7) == 0) f.launch_at = std::atol(e + 7);
+            if (std::strcmp(e, "exchange") == 0) f.exchange = true;
+        }
+#endif
+        return f;
+    }();
+    return plan;
+}
+
+// The grid of a launch: `g`, or an empty grid for the launch fault injection
+// picks (one count over every launcher of the process).
+#ifdef WKV4_CHECKED
+static std::atomic<long> g_launches{0};
+#endif
+template <typename G>
+static G launch_grid(G g) {
+#ifdef WKV4_CHECKED
+    const long at = fault_plan().launch_at;
+    if (at > 0 && g_launches.fetch_add(1) + 1 == at) return G(0);
+#endif
+    return g;
+}
+
+static const ScanOverrides& scan_overrides() {
+    static const ScanOverrides o{env_int("WKV4_SCAN_NW", 0), env_int("WKV4_SCAN_CLUSTER", 0),
+                                 env_int("WKV4_SCAN_WAVES", 0)};
+    return o;
+}
+
+// Dynamic shared memory to request for a scan CTA of `cta_regs` registers
+// (its warps' allocations) that holds `cols` tensor-memory columns.  A CTA
+// allocates its columns at its start and holds them to its end, and an
+// allocation that cannot be met waits for another CTA's release; so every
+// set of scan CTAs an SM can hold at once -- of one call or of concurrent
+// calls on other streams, of any dtypes and shapes -- must need at most the
+// SM's 512 columns.  It does when each scan CTA takes at least its column
+// share (cols / 512) of one resource the SM divides among its CTAs: its
+// registers (cta_regs >= reg_file * cols / 512, true of every 8-warp scan at
+// the 128-register cap and 256 columns or fewer), else shared memory, whose
+// request is then raised to per_sm * cols / 512 (less the per-block
+// reservation).  Either way no scan CTA's allocation waits on another's.
+static size_t scan_smem_request(size_t bytes, int cols, int cta_regs) {
+    const DeviceAttrs& at = device_attrs();
+    if ((int64_t)cta_regs * kTmemColumns >= (int64_t)at.reg_file * cols) return bytes;
+    const size_t share = ((size_t)at.smem_per_sm * (size_t)cols + kTmemColumns - 1) / kTmemColumns;
+    size_t need = share > (size_t)at.smem_reserved ? share - (size_t)at.smem_reserved : 0;
     need = (need + 127) & ~(size_t)127;
     return bytes > need ? bytes : need;
 }
@@ -137,12 +232,10 @@ static cudaError_t clusters_fit(int nwi, int nc, int bps, int& out) {
     int v = slot.load(std::memory_order_acquire);
     if (v == 0) {
         if ((e = ensure_smem_attr(attr, wkv4_occupancy_stand_in, kMaxSmem)) != cudaSuccess) return e;
-        int per_sm = 233472, reserved = 1024;
-        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+        const DeviceAttrs& da = device_attrs();
         // the request at which bps, and not bps + 1, CTAs fit on an SM
-        size_t req = (size_t)per_sm / (size_t)(bps + 1) + 1;
-        req = req > (size_t)reserved ? req - (size_t)reserved : 0;
+        size_t req = (size_t)da.smem_per_sm / (size_t)(bps + 1) + 1;
+        req = req > (size_t)da.smem_reserved ? req - (size_t)da.smem_reserved : 0;
         if (req > kMaxSmem) req = kMaxSmem;
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof(cfg));
@@ -171,39 +264,45 @@ static cudaError_t clusters_fit(int nwi, int nc, int bps, int& out) {
 // memory cap may have raised), threads and tensor-memory columns.  Worked out
 // here rather than asked of the runtime, whose per-SM occupancy query
 // reports one CTA for these kernels where the SM holds two.
-template <typename IO, int L, bool kMulti, bool kTMA>
-static cudaError_t scan_ctas_per_sm(int nw, int nc, int& bps) {
+// Registers a thread of one scan instantiation uses (queried once per device;
+// the dynamic shared-memory limit is raised with it).
+template <typename IO, int L, bool kMulti, bool kTMA, bool kGate>
+static cudaError_t scan_regs(int& regs) {
     static DeviceFlags attr;
-    static std::atomic<int> regs_cache[64];
-    bps = 0;
-    auto kern = wkv4_scan_kernel<IO, L, kMulti, kTMA>;
+    static std::atomic<int> regs_cache[kMaxDevices];
+    auto kern = wkv4_scan_kernel<IO, L, kMulti, kTMA, kGate>;
     cudaError_t e = ensure_smem_attr(attr, kern, kMaxSmem);
     if (e != cudaSuccess) return e;
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    int regs = regs_cache[dev].load(std::memory_order_acquire);
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    regs = regs_cache[dev].load(std::memory_order_acquire);
     if (regs == 0) {
         cudaFuncAttributes fa;
         if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
         regs = fa.numRegs > 0 ? fa.numRegs : 1;
         regs_cache[dev].store(regs, std::memory_order_release);
     }
+    return cudaSuccess;
+}
+
+static int warp_regs(int regs) { return ((regs * 32 + 255) / 256) * 256; }  // allocated in 256s
+
+template <typename IO, int L, bool kMulti, bool kTMA, bool kGate>
+static cudaError_t scan_ctas_per_sm(int nw, int nc, int& bps) {
+    bps = 0;
+    int regs = 0;
+    cudaError_t e = scan_regs<IO, L, kMulti, kTMA, kGate>(regs);
+    if (e != cudaSuccess) return e;
     const ScanLayout<IO, L, kMulti> lay{nw, nc};
-    const size_t req = scan_smem_request(lay.bytes(), lay.tmem_cols());
+    const size_t req = scan_smem_request(lay.bytes(), lay.tmem_cols(), warp_regs(regs) * nw);
     if (req > kMaxSmem || lay.tmem_cols() > kTmemColumns) return cudaSuccess;
-    int per_sm = 233472, reserved = 1024, reg_file = 65536, max_thr = 2048, max_blk = 32;
-    cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
-    cudaDeviceGetAttribute(&reg_file, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
-    cudaDeviceGetAttribute(&max_thr, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
-    cudaDeviceGetAttribute(&max_blk, cudaDevAttrMaxBlocksPerMultiprocessor, dev);
-    const int warp_regs = ((regs * 32 + 255) / 256) * 256;  // allocated per warp in 256s
-    int n = reg_file / (warp_regs * nw);
-    n = std::min(n, (int)((size_t)per_sm / (req + (size_t)reserved)));
-    n = std::min(n, max_thr / (32 * nw));
+    const DeviceAttrs& at = device_attrs();
+    int n = at.reg_file / (warp_regs(regs) * nw);
+    n = std::min(n, (int)((size_t)at.smem_per_sm / (req + (size_t)at.smem_reserved)));
+    n = std::min(n, at.max_threads / (32 * nw));
     n = std::min(n, kTmemColumns / lay.tmem_cols());
-    n = std::min(n, max_blk);
+    n = std::min(n, at.max_blocks);
     bps = n > 0 ? n : 0;
     return cudaSuccess;
 }
@@ -222,9 +321,9 @@ struct ScanShape {
     int64_t clusters;
 };
 
-template <typename IO, int L, bool kTMA>
+template <typename IO, int L, bool kTMA, bool kGate>
 static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
-    const int force_nw = env_int("WKV4_SCAN_NW", 0), force_nc = env_int("WKV4_SCAN_CLUSTER", 0);
+    const int force_nw = scan_overrides().nw, force_nc = scan_overrides().nc;
     cudaError_t e = cudaSuccess;
     for (int i = 0; i < 2; ++i) {
         const int nw = kNwChoices[i];
@@ -238,7 +337,8 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
         } else {
             for (int c = kMaxCluster; c > 1; c /= 2) {
                 int bps = 0, fit = 0;
-                if ((e = scan_ctas_per_sm<IO, L, true, kTMA>(nw, c, bps)) != cudaSuccess) return e;
+                if ((e = scan_ctas_per_sm<IO, L, true, kTMA, kGate>(nw, c, bps)) != cudaSuccess)
+                    return e;
                 if ((e = clusters_fit(i, c, bps, fit)) != cudaSuccess) return e;
                 if ((int64_t)fit >= tiles) {
                     nc = c;
@@ -249,12 +349,12 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
         const int64_t rounds = (nseg + nc - 1) / nc;
         if (rounds > (1ll << 30)) continue;
         int bps = 0;
-        e = rounds == 1 ? scan_ctas_per_sm<IO, L, false, kTMA>(nw, nc, bps)
-                        : scan_ctas_per_sm<IO, L, true, kTMA>(nw, nc, bps);
+        e = rounds == 1 ? scan_ctas_per_sm<IO, L, false, kTMA, kGate>(nw, nc, bps)
+                        : scan_ctas_per_sm<IO, L, true, kTMA, kGate>(nw, nc, bps);
         if (e != cudaSuccess) return e;
         if (bps <= 0) continue;  // does not fit on an SM
         int64_t clusters = tiles;
-        if (rounds == 1 && !env_int("WKV4_SCAN_WAVES", 0)) {
+        if (rounds == 1 && !scan_overrides().waves) {
             int fit = 0;
             if ((e = clusters_fit(i, nc, bps, fit)) != cudaSuccess) return e;
             if (fit > 0 && fit < tiles) clusters = fit;
@@ -265,26 +365,31 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
     return cudaErrorInvalidConfiguration;
 }
 
-template <typename IO, int L, bool kMulti, bool kTMA>
+template <typename IO, int L, bool kMulti, bool kTMA, bool kGate>
 static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const ScanShape& sh,
                                   EncodeFn encode) {
-    CUtensorMap tk, tv, ty;
+    CUtensorMap tk, tv, ty, tr;
     std::memset(&tk, 0, sizeof(tk));
     std::memset(&tv, 0, sizeof(tv));
     std::memset(&ty, 0, sizeof(ty));
+    std::memset(&tr, 0, sizeof(tr));
     if (kTMA) {
         if (!encode(&tk, a.k, a.dtype, a.B, a.T, a.C, 64, L) ||
             !encode(&tv, a.v, a.dtype, a.B, a.T, a.C, 64, L) ||
-            !encode(&ty, a.y, a.dtype, a.B, a.T, a.C, 64, L))
+            !encode(&ty, a.y, a.dtype, a.B, a.T, a.C, 64, L) ||
+            (kGate && !encode(&tr, a.r, a.dtype, a.B, a.T, a.C, 64, L)))
             return cudaErrorInvalidValue;
     }
-    auto kern = wkv4_scan_kernel<IO, L, kMulti, kTMA>;
+    auto kern = wkv4_scan_kernel<IO, L, kMulti, kTMA, kGate>;
     const ScanLayout<IO, L, kMulti> lay{sh.nw, sh.nc};
+    int regs = 0;
+    cudaError_t e = scan_regs<IO, L, kMulti, kTMA, kGate>(regs);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)(sh.clusters * sh.nc), 1, 1);
+    cfg.gridDim = dim3(launch_grid((unsigned)(sh.clusters * sh.nc)), 1, 1);
     cfg.blockDim = dim3(32 * sh.nw, 1, 1);
-    cfg.dynamicSmemBytes = scan_smem_request(lay.bytes(), lay.tmem_cols());
+    cfg.dynamicSmemBytes = scan_smem_request(lay.bytes(), lay.tmem_cols(), warp_regs(regs) * sh.nw);
     cfg.stream = a.stream;
     cudaLaunchAttribute attrs[1];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
@@ -293,10 +398,10 @@ static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const S
     attrs[0].val.clusterDim.z = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tk, tv, ty, p);
+    return cudaLaunchKernelEx(&cfg, kern, tk, tv, ty, tr, p);
 }
 
-template <typename IO, bool kTMA>
+template <typename IO, bool kTMA, bool kGate>
 static cudaError_t launch_scan_t(const FwdArgs& a, EncodeFn encode) {
     constexpr int L = ScanL<IO>::L;
     ScanParams p{};
@@ -307,40 +412,46 @@ static cudaError_t launch_scan_t(const FwdArgs& a, EncodeFn encode) {
     p.u = a.u;
     p.k = a.k;
     p.v = a.v;
+    p.r = a.r;
     p.state_in = a.state_in;
     p.y = a.y;
     p.state_out = a.state_out;
     p.BC = a.B * a.C;
+    p.wait_rounds = wait_rounds();
+    p.no_push = fault_plan().exchange ? 1 : 0;
     p.bulk_params = ((uintptr_t)a.w % 16 == 0) && ((uintptr_t)a.u % 16 == 0) &&
                     ((uintptr_t)a.state_in % 16 == 0) && (a.C % 4 == 0);
     const int64_t tiles = a.B * p.CGB;
     if (tiles > (1ll << 30)) return cudaErrorInvalidConfiguration;
     ScanShape sh;
-    cudaError_t e = pick_scan_shape<IO, L, kTMA>(tiles, a.T, sh);
+    cudaError_t e = pick_scan_shape<IO, L, kTMA, kGate>(tiles, a.T, sh);
     if (e != cudaSuccess) return e;
     if (sh.clusters * sh.nc > (int64_t)INT32_MAX) return cudaErrorInvalidConfiguration;
     p.tiles = (int)tiles;
     p.rounds = sh.rounds;
-    if (sh.rounds == 1) return launch_scan_nb<IO, L, false, kTMA>(a, p, sh, encode);
-    return launch_scan_nb<IO, L, true, kTMA>(a, p, sh, encode);
+    if (sh.rounds == 1) return launch_scan_nb<IO, L, false, kTMA, kGate>(a, p, sh, encode);
+    return launch_scan_nb<IO, L, true, kTMA, kGate>(a, p, sh, encode);
+}
+
+template <typename IO>
+static cudaError_t launch_scan_io(const FwdArgs& a, bool tma, EncodeFn encode) {
+    if (a.r) return tma ? launch_scan_t<IO, true, true>(a, encode) : launch_scan_t<IO, false, true>(a, encode);
+    return tma ? launch_scan_t<IO, true, false>(a, encode) : launch_scan_t<IO, false, false>(a, encode);
 }
 
 cudaError_t launch_scan(const FwdArgs& a, bool tma, EncodeFn encode) {
     switch (a.dtype) {
-        case WKV4_F32:
-            return tma ? launch_scan_t<float, true>(a, encode) : launch_scan_t<float, false>(a, encode);
-        case WKV4_F16:
-            return tma ? launch_scan_t<__half, true>(a, encode) : launch_scan_t<__half, false>(a, encode);
-        default:
-            return tma ? launch_scan_t<__nv_bfloat16, true>(a, encode)
-                       : launch_scan_t<__nv_bfloat16, false>(a, encode);
+        case WKV4_F32: return launch_scan_io<float>(a, tma, encode);
+        case WKV4_F16: return launch_scan_io<__half>(a, tma, encode);
+        default: return launch_scan_io<__nv_bfloat16>(a, tma, encode);
     }
 }
 
-template <typename IO, int L, int NW, int NS>
-static cudaError_t launch_seq_t(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv) {
+template <typename IO, int L, int NW, int NS, bool kGate>
+static cudaError_t launch_seq_g(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
+                                const CUtensorMap* tr) {
     using Sh = SeqShape<IO, L, NW, NS>;
-    auto kern = wkv4_seq_kernel<IO, L, NW, NS>;
+    auto kern = wkv4_seq_kernel<IO, L, NW, NS, kGate>;
     static DeviceFlags attr;
     cudaError_t e = ensure_smem_attr(attr, kern, Sh::kSmem);
     if (e != cudaSuccess) return e;
@@ -350,20 +461,30 @@ static cudaError_t launch_seq_t(const FwdArgs& a, const CUtensorMap* tk, const C
     p.CGB = (int)((a.C + Sh::kCw - 1) / Sh::kCw);
     p.w = a.w;
     p.u = a.u;
+    p.r = a.r;
     p.state_in = a.state_in;
     p.y = a.y;
     p.state_out = a.state_out;
     p.BC = a.B * a.C;
+    p.wait_rounds = wait_rounds();
     const int64_t grid = a.B * p.CGB;
-    kern<<<(unsigned)grid, Sh::kThreads, Sh::kSmem, a.stream>>>(*tk, *tv, p);
+    kern<<<launch_grid((unsigned)grid), Sh::kThreads, Sh::kSmem, a.stream>>>(*tk, *tv, *tr, p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_seq(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv) {
+template <typename IO, int L, int NW, int NS>
+static cudaError_t launch_seq_t(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
+                                const CUtensorMap* tr) {
+    return a.r ? launch_seq_g<IO, L, NW, NS, true>(a, tk, tv, tr)
+               : launch_seq_g<IO, L, NW, NS, false>(a, tk, tv, tk);
+}
+
+cudaError_t launch_seq(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
+                       const CUtensorMap* tr) {
     switch (a.dtype) {
-        case WKV4_F32: return launch_seq_t<WKV4_SEQ_F32>(a, tk, tv);
-        case WKV4_F16: return launch_seq_t<WKV4_SEQ_F16>(a, tk, tv);
-        default: return launch_seq_t<WKV4_SEQ_BF16>(a, tk, tv);
+        case WKV4_F32: return launch_seq_t<WKV4_SEQ_F32>(a, tk, tv, tr);
+        case WKV4_F16: return launch_seq_t<WKV4_SEQ_F16>(a, tk, tv, tr);
+        default: return launch_seq_t<WKV4_SEQ_BF16>(a, tk, tv, tr);
     }
 }
 
@@ -379,7 +500,16 @@ static StepParams step_params(const FwdArgs& a) {
     p.state_in = a.state_in;
     p.y = a.y;
     p.state_out = a.state_out;
+    p.r = a.r;
     return p;
+}
+
+template <typename IO>
+static void launch_step_io(const FwdArgs& a, const StepParams& p, unsigned grid) {
+    if (a.r)
+        wkv4_step_kernel<IO, true><<<launch_grid(grid), 256, 0, a.stream>>>(p);
+    else
+        wkv4_step_kernel<IO, false><<<launch_grid(grid), 256, 0, a.stream>>>(p);
 }
 
 cudaError_t launch_step(const FwdArgs& a) {
@@ -387,9 +517,9 @@ cudaError_t launch_step(const FwdArgs& a) {
     const int64_t BC = a.B * a.C;
     const unsigned grid = (unsigned)((BC + 255) / 256);
     switch (a.dtype) {
-        case WKV4_F32: wkv4_step_kernel<float><<<grid, 256, 0, a.stream>>>(p); break;
-        case WKV4_F16: wkv4_step_kernel<__half><<<grid, 256, 0, a.stream>>>(p); break;
-        default: wkv4_step_kernel<__nv_bfloat16><<<grid, 256, 0, a.stream>>>(p); break;
+        case WKV4_F32: launch_step_io<float>(a, p, grid); break;
+        case WKV4_F16: launch_step_io<__half>(a, p, grid); break;
+        default: launch_step_io<__nv_bfloat16>(a, p, grid); break;
     }
     return cudaGetLastError();
 }
@@ -398,20 +528,28 @@ static bool aligned(const void* ptr, size_t bytes) {
     return ptr == nullptr || ((uintptr_t)ptr % bytes) == 0;
 }
 
+template <typename IO, int V>
+static void launch_decode_io(const FwdArgs& a, const StepParams& p, unsigned grid) {
+    if (a.r)
+        wkv4_decode_kernel<IO, V, false, true><<<launch_grid(grid), 256, 0, a.stream>>>(p);
+    else
+        wkv4_decode_kernel<IO, V, false, false><<<launch_grid(grid), 256, 0, a.stream>>>(p);
+}
+
 cudaError_t launch_decode(const FwdArgs& a) {
     constexpr int V = 4;
     const size_t es = dtype_size(a.dtype);
     const bool vec = (a.C % V == 0) && aligned(a.k, V * es) && aligned(a.v, V * es) &&
-                     aligned(a.y, V * es) && aligned(a.w, 16) && aligned(a.u, 16) &&
-                     aligned(a.state_in, 16) && aligned(a.state_out, 16);
+                     aligned(a.r, V * es) && aligned(a.y, V * es) && aligned(a.w, 16) &&
+                     aligned(a.u, 16) && aligned(a.state_in, 16) && aligned(a.state_out, 16);
     if (!vec) return launch_step(a);
     const StepParams p = step_params(a);
     const int64_t threads = a.B * a.C / V;
     const unsigned grid = (unsigned)((threads + 255) / 256);
     switch (a.dtype) {
-        case WKV4_F32: wkv4_decode_kernel<float, V><<<grid, 256, 0, a.stream>>>(p); break;
-        case WKV4_F16: wkv4_decode_kernel<__half, V><<<grid, 256, 0, a.stream>>>(p); break;
-        default: wkv4_decode_kernel<__nv_bfloat16, V><<<grid, 256, 0, a.stream>>>(p); break;
+        case WKV4_F32: launch_decode_io<float, V>(a, p, grid); break;
+        case WKV4_F16: launch_decode_io<__half, V>(a, p, grid); break;
+        default: launch_decode_io<__nv_bfloat16, V>(a, p, grid); break;
     }
     return cudaGetLastError();
 }
@@ -429,15 +567,15 @@ cudaError_t launch_decode_slots(const FwdArgs& a, const int32_t* slots, int64_t 
     const unsigned grid = (unsigned)((threads + 255) / 256);
     if (vec) {
         switch (a.dtype) {
-            case WKV4_F32: wkv4_decode_kernel<float, V, true><<<grid, 256, 0, a.stream>>>(p); break;
-            case WKV4_F16: wkv4_decode_kernel<__half, V, true><<<grid, 256, 0, a.stream>>>(p); break;
-            default: wkv4_decode_kernel<__nv_bfloat16, V, true><<<grid, 256, 0, a.stream>>>(p); break;
+            case WKV4_F32: wkv4_decode_kernel<float, V, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            case WKV4_F16: wkv4_decode_kernel<__half, V, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            default: wkv4_decode_kernel<__nv_bfloat16, V, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
         }
     } else {
         switch (a.dtype) {
-            case WKV4_F32: wkv4_decode_kernel<float, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
-            case WKV4_F16: wkv4_decode_kernel<__half, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
-            default: wkv4_decode_kernel<__nv_bfloat16, 1, true><<<grid, 256, 0, a.stream>>>(p); break;
+            case WKV4_F32: wkv4_decode_kernel<float, 1, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            case WKV4_F16: wkv4_decode_kernel<__half, 1, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            default: wkv4_decode_kernel<__nv_bfloat16, 1, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
         }
     }
     return cudaGetLastError();
@@ -464,15 +602,15 @@ cudaError_t launch_token_shift(const ShiftArgs& a) {
                     (unsigned)a.B);
     if (vec) {
         switch (a.dtype) {
-            case WKV4_F32: wkv4_token_shift_kernel<float, 4><<<grid, 256, 0, a.stream>>>(p); break;
-            case WKV4_F16: wkv4_token_shift_kernel<__half, 8><<<grid, 256, 0, a.stream>>>(p); break;
-            default: wkv4_token_shift_kernel<__nv_bfloat16, 8><<<grid, 256, 0, a.stream>>>(p); break;
+            case WKV4_F32: wkv4_token_shift_kernel<float, 4><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            case WKV4_F16: wkv4_token_shift_kernel<__half, 8><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            default: wkv4_token_shift_kernel<__nv_bfloat16, 8><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
         }
     } else {
         switch (a.dtype) {
-            case WKV4_F32: wkv4_token_shift_kernel<float, 1><<<grid, 256, 0, a.stream>>>(p); break;
-            case WKV4_F16: wkv4_token_shift_kernel<__half, 1><<<grid, 256, 0, a.stream>>>(p); break;
-            default: wkv4_token_shift_kernel<__nv_bfloat16, 1><<<grid, 256, 0, a.stream>>>(p); break;
+            case WKV4_F32: wkv4_token_shift_kernel<float, 1><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            case WKV4_F16: wkv4_token_shift_kernel<__half, 1><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            default: wkv4_token_shift_kernel<__nv_bfloat16, 1><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
         }
     }
     return cudaGetLastError();
@@ -481,8 +619,16 @@ cudaError_t launch_token_shift(const ShiftArgs& a) {
 cudaError_t launch_copy_state(const FwdArgs& a) {
     const int64_t BC = a.B * a.C;
     if (!a.state_out || BC == 0) return cudaSuccess;
-    wkv4_copy_state_kernel<<<(unsigned)((BC + 255) / 256), 256, 0, a.stream>>>(a.state_in,
+    wkv4_copy_state_kernel<<<launch_grid((unsigned)((BC + 255) / 256)), 256, 0, a.stream>>>(a.state_in,
                                                                                a.state_out, BC);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_combine(int64_t B, int64_t C, const float* w, int64_t n, const float* x,
+                                 const float* y, float* out, cudaStream_t stream) {
+    const int64_t BC = B * C;
+    wkv4_state_combine_kernel<<<launch_grid((unsigned)((BC + 255) / 256)), 256, 0, stream>>>(
+        w, n, x, y, out, B, C);
     return cudaGetLastError();
 }
 

@@ -94,11 +94,14 @@ struct ScanLayout {
     __host__ __device__ size_t params(int slot) const {  // [kParamSlots][5][Cg] f32
         return agg(kAggSlots) + (size_t)slot * 5 * kCg * 4;
     }
-    // rows [nw], params [kParamSlots], aggregate slots [kAggSlots] x 8 B
+    // rows [nw], params [kParamSlots], aggregate slots [kAggSlots], receptance
+    // rows [nw] x 8 B
     __host__ __device__ size_t bars() const { return params(kParamSlots); }
     __host__ __device__ size_t tslot() const {
-        return bars() + (size_t)(nw + kParamSlots + kAggSlots) * 8;
+        return bars() + (size_t)(2 * nw + kParamSlots + kAggSlots) * 8;
     }
+    // the CTA's failure flag (a bounded wait ran out), beside the tensor-memory base
+    __host__ __device__ size_t flag() const { return tslot() + 4; }
     __host__ __device__ size_t bytes() const { return kAlign + tslot() + 8; }
     // tensor-memory columns: 4 a step for each warp and slot, warps w and
     // w + 4 sharing a lane quarter
@@ -114,11 +117,14 @@ struct ScanParams {
     const float* u;
     const void* k;
     const void* v;
+    const void* r;        // receptance [B][T][C] of the gated forward (kGate), else NULL
     const float* state_in;
     void* y;
     float* state_out;
     int64_t BC;
-    int bulk_params;  // w, u, state_in 16-byte aligned and C % 4 == 0: bulk copies
+    int bulk_params;      // w, u, state_in 16-byte aligned and C % 4 == 0: bulk copies
+    uint32_t wait_rounds;  // limit of each bounded wait, in rounds of about 1 ms
+    int no_push;           // checked builds only: no CTA pushes its aggregate (fault injection)
 };
 
 // (a, b, p) triples in shared memory, stored as three planes of n entries.
@@ -227,10 +233,18 @@ __device__ __forceinline__ void fold_aggs(const TripleRef& agg, int col, int ran
     }
 }
 
-template <typename IO, int L, bool kMulti, bool kTMA>
+// kGate: the gated forward, y = sigmoid(r) wkv (the receptance gate of the
+// time mix applied in the output pass).  With one round and TMA the warp's r
+// rows come by their own TMA box (on their own barrier) into its v rows once
+// the summary pass has read them, and y is written over them in place; with
+// several rounds or element-wise loads r is read from global memory in the
+// output pass (several rounds: the warp's r box is prefetched into L2 at its
+// summary pass).
+template <typename IO, int L, bool kMulti, bool kTMA, bool kGate>
 __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     wkv4_scan_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                     const __grid_constant__ CUtensorMap tmy, const ScanParams p) {
+                     const __grid_constant__ CUtensorMap tmy, const __grid_constant__ CUtensorMap tmr,
+                     const ScanParams p) {
     using Lay = ScanLayout<IO, L, kMulti>;
     constexpr int kAS = Lay::kAggSlots;
     constexpr int Cg = Lay::kCg;
@@ -248,6 +262,7 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     uint64_t* mbar = reinterpret_cast<uint64_t*>(base + lay.bars());  // rows [NW]
     uint64_t* pbar = mbar + NW;                                       // params [kParamSlots]
     uint64_t* abar = pbar + Lay::kParamSlots;  // [kAS]: the aggregates of a round have landed
+    uint64_t* rbar = abar + kAS;               // [NW]: a warp's receptance rows (kGate)
     uint32_t* tslot = reinterpret_cast<uint32_t*>(base + lay.tslot());
 
     const int rank = (int)cluster.block_rank();
@@ -259,8 +274,14 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int col = lane * 2;
     const int64_t seg_stride = (int64_t)NC * Ts;  // steps per round
+    const int64_t BTC = p.BC * T, Bn = p.BC / C;  // extents of k, v, y (and r); batch rows
+    // a TMA box's start inside its [B][T][C] tensor (checked builds)
+    auto box_in = [&](int64_t cc0, int64_t t, int64_t bb) {
+        return in_range(cc0, C) && in_range(t, T) && in_range(bb, Bn);
+    };
     const IO* kg = static_cast<const IO*>(p.k);
     const IO* vg = static_cast<const IO*>(p.v);
+    const IO* rg = static_cast<const IO*>(p.r);
     IO* yg = static_cast<IO*>(p.y);
     // aggregate exchanges this cluster makes: one a round, or one a tile
     const int items = kMulti ? p.rounds : (p.tiles - tile + G - 1) / G;
@@ -273,13 +294,19 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     IO* const vr = reinterpret_cast<IO*>(base + lay.v()) + warp * L * Cg;
     // Lane 0 of each warp: this warp's rows of round j of the tile at (bb,
     // cc0), k and v (issue_k announces both on the warp's barrier, issue_v may
-    // follow later).  Every round completes one phase of the barrier (a plain
-    // arrive where nothing is copied), so its phases stay in step.
-    auto issue_k = [&](int j, int bb, int64_t cc0) {
+    // follow later), as the barrier's phase `phase` (the tile with one round,
+    // the round with several).  Every round completes one phase of the
+    // barrier (a plain arrive where nothing is copied), so its phases stay in
+    // step; row_pend records the phase issued and not yet waited for (-1:
+    // none; a wait is always for the last phase issued), so that a CTA
+    // leaving after an expired wait can let a copy in flight land.
+    int row_pend = -1;
+    auto issue_k = [&](int j, int bb, int64_t cc0, int phase) {
         if constexpr (kTMA) {
+            row_pend = phase;
             uint64_t* bar = mbar + warp;
-            if (chunk_len(j, warp) > 0) {
-                const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
+            const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
+            if (chunk_len(j, warp) > 0 && box_in(cc0, t, bb)) {
                 mbar_arrive_expect_tx(bar, 2u * kChunkBytes);
                 tma_load_3d(kr, &tmk, (int)cc0, t, bb, bar);
             } else {
@@ -289,31 +316,49 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     };
     auto issue_v = [&](int j, int bb, int64_t cc0) {
         if constexpr (kTMA) {
-            if (chunk_len(j, warp) > 0) {
-                const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
+            const int t = (int)((int64_t)j * seg_stride + (int64_t)rank * Ts + warp * L);
+            if (chunk_len(j, warp) > 0 && box_in(cc0, t, bb))
                 tma_load_3d(vr, &tmv, (int)cc0, t, bb, mbar + warp);
-            }
         }
     };
-    auto issue_rows = [&](int j, int bb, int64_t cc0) {
-        issue_k(j, bb, cc0);
+    auto issue_rows = [&](int j, int bb, int64_t cc0, int phase) {
+        issue_k(j, bb, cc0, phase);
         issue_v(j, bb, cc0);
+    };
+    // Lane 0, one round with TMA and the gate: this warp's r rows of the tile
+    // at (bb, cc0) into its v rows, as phase `phase` (the tile) of its
+    // receptance barrier (a plain arrive where nothing is copied).
+    int r_pend = -1;
+    auto issue_r = [&](int bb, int64_t cc0, int phase) {
+        if constexpr (kTMA && kGate && !kMulti) {
+            r_pend = phase;
+            const int t = (int)((int64_t)rank * Ts + warp * L);
+            if (chunk_len(0, warp) > 0 && box_in(cc0, t, bb)) {
+                mbar_arrive_expect_tx(rbar + warp, (uint32_t)kChunkBytes);
+                tma_load_3d(vr, &tmr, (int)cc0, t, bb, rbar + warp);
+            } else {
+                mbar_arrive(rbar + warp);
+            }
+        }
     };
     // Per-channel w, u and the state of a tile: a full 64-channel slice with
     // aligned pointers comes by bulk copy (lane 0 of warp 0) into a parameter
     // slot, on that slot's barrier; any other tile (read from global memory
     // by take_params) completes the slot's phase by a plain arrive, so that
     // every tile takes exactly one phase of its slot and the waits' parities
-    // stay in step with the tiles.
+    // stay in step with the tiles.  par_pend (lane 0 of warp 0): the tile
+    // whose parameters were issued and not yet waited for (-1: none).
+    int par_pend = -1;
     auto bulk_ok = [&](int64_t cc0) { return kTMA && p.bulk_params && cc0 + Cg <= C; };
-    auto issue_params = [&](int slot, int bb, int64_t cc0) {
-        if (!bulk_ok(cc0)) {
+    auto issue_params = [&](int slot, int bb, int64_t cc0, int tile_no) {
+        par_pend = tile_no;
+        const int64_t ch = (int64_t)bb * C + cc0;
+        if (!bulk_ok(cc0) || !(in_range(cc0 + Cg - 1, C) && in_range(ch + Cg - 1, p.BC))) {
             mbar_arrive(pbar + slot);
             return;
         }
         float* sw = reinterpret_cast<float*>(base + lay.params(slot));
         const uint32_t nb = Cg * 4;
-        const int64_t ch = (int64_t)bb * C + cc0;
         mbar_arrive_expect_tx(pbar + slot, (p.state_in ? 5u : 2u) * nb);
         bulk_load(sw, p.w + cc0, nb, pbar + slot);
         bulk_load(sw + Cg, p.u + cc0, nb, pbar + slot);
@@ -324,9 +369,20 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
         }
     };
 
-    // every CTA of the cluster pushes 32 B per lane into each aggregate slot
+    // every CTA of the cluster pushes 32 B per lane into each aggregate slot;
+    // agg_waited (warp 1): the exchanges whose aggregates it has seen land, in
+    // order; slots are armed for exchanges agg_waited .. agg_waited + kAS - 1
+    // (those below `items`)
     const uint32_t agg_bytes = (uint32_t)NC * 32u * 32u;
+    int agg_waited = 0;
+    // The CTA's failure flag: set by any thread whose bounded wait ran out.
+    // From then on the CTA issues no copy, pushes no aggregate and waits on no
+    // barrier (outputs and final state are then undefined, and the device
+    // error word says so); before leaving it lets the copies it issued, and
+    // the aggregates its slots were armed for, land (bounded waits).
+    volatile int* s_fail = reinterpret_cast<volatile int*>(base + lay.flag());
     if (threadIdx.x == 0) {
+        *s_fail = 0;
         for (int r = 0; r < kAS; ++r) mbar_init(abar + r, 1);
         fence_mbar_init();
         for (int r = 0; r < kAS && r < items; ++r) mbar_arrive_expect_tx(abar + r, agg_bytes);
@@ -338,11 +394,13 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
                 prefetch_tmap(&tmk);
                 prefetch_tmap(&tmv);
                 prefetch_tmap(&tmy);
+                if (kGate) prefetch_tmap(&tmr);
             }
             mbar_init(mbar + warp, 1);
+            if (kGate) mbar_init(rbar + warp, 1);
             fence_mbar_init();
-            if (warp == 0) issue_params(0, b, c0);
-            issue_rows(0, b, c0);
+            if (warp == 0) issue_params(0, b, c0, 0);
+            issue_rows(0, b, c0, 0);
         }
         __syncwarp();
     }
@@ -362,18 +420,32 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     auto taddr = [&](int s) -> uint32_t {
         return tbase + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(s * NW * L + (warp >> 2) * 4 * L);
     };
+    // this thread has seen the CTA fail: its own wait ran out, or the flag
+    // was set when it last passed a CTA barrier (other warps learn of a
+    // failure there; until then their copies are tracked and their waits
+    // bounded as on the normal path)
     bool failed = false;
+    auto cta_failed = [&]() -> bool { return failed; };
+    auto sync_fail = [&]() { failed = failed || *s_fail != 0; };
+    auto fail = [&](unsigned bit) {
+        failed = true;
+        *s_fail = 1;
+        if (lane == 0) atomicOr(&g_device_error, bit);
+    };
 
     // w, u of the current tile (cc) and the state carried into it (carry;
     // only warp 1 folds it), from parameter slot `slot` (its phase `parity`)
     // or, for a partial or unaligned slice, from global memory
     PairConsts cc;
     St carry[2];
-    auto take_params = [&](int slot, uint32_t parity) {
+    auto take_params = [&](int slot, uint32_t parity, int tile_no) {
         if (bulk_ok(c0)) {
-            if (!failed && !mbar_wait_bounded(pbar + slot, parity)) {
-                failed = true;
-                if (lane == 0) atomicOr(&g_device_error, kErrTmaWait);
+            if (!cta_failed()) {
+                if (mbar_wait_bounded(pbar + slot, parity, p.wait_rounds)) {
+                    if (par_pend == tile_no) par_pend = -1;
+                } else {
+                    fail(kErrTmaWait);
+                }
             }
             const float* sw = reinterpret_cast<const float*>(base + lay.params(slot));
 #pragma unroll
@@ -388,9 +460,10 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
             pair_wu(p.w, p.u, c0 + col, C, cc);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int64_t c = c0 + col + j;
-                carry[j] = (p.state_in && c < C) ? load_state_log2(p.state_in, p.BC, (int64_t)b * C + c)
-                                                 : empty_state();
+                const int64_t c = c0 + col + j, ch = (int64_t)b * C + c;
+                carry[j] = (p.state_in && c < C && in_range(ch, p.BC))
+                               ? load_state_log2(p.state_in, p.BC, ch)
+                               : empty_state();
             }
         }
         pair_derive(cc);
@@ -399,8 +472,8 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
         if (rank == 0 && warp == 1 && p.state_out) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int64_t c = c0 + col + j;
-                if (c < C) store_state_log2(p.state_out, p.BC, (int64_t)b * C + c, carry[j]);
+                const int64_t c = c0 + col + j, ch = (int64_t)b * C + c;
+                if (c < C && in_range(ch, p.BC)) store_state_log2(p.state_out, p.BC, ch, carry[j]);
             }
         }
     };
@@ -409,14 +482,17 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     //         entry of summary slot round & 1 (kMulti) and its stash into
     //         tensor-memory slot round & 1, once its rows (barrier phase
     //         `parity`) are in
-    auto summary = [&](int round, uint32_t parity) -> PairRef {
+    auto summary = [&](int round, int phase) -> PairRef {
         const int slot = kMulti ? (round & 1) : 0;
         const int n = chunk_len(round, warp);
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;  // segment start
         if constexpr (kTMA) {
-            if (n > 0 && !failed && !mbar_wait_bounded(mbar + warp, parity)) {
-                failed = true;
-                if (lane == 0) atomicOr(&g_device_error, kErrTmaWait);
+            if (n > 0 && !cta_failed()) {
+                if (mbar_wait_bounded(mbar + warp, (uint32_t)(phase & 1), p.wait_rounds)) {
+                    if (row_pend == phase) row_pend = -1;
+                } else {
+                    fail(kErrTmaWait);
+                }
             }
         } else {
             // element-wise loads of this warp's rows (any alignment, zero fill)
@@ -426,13 +502,20 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
                 IO kx = Io<IO>::from_f(0.f), vx = Io<IO>::from_f(0.f);
                 if (t < T && c < C) {
                     const int64_t off = ((int64_t)b * T + t) * C + c;
-                    kx = kg[off];
-                    vx = vg[off];
+                    if (in_range(off, BTC)) {
+                        kx = kg[off];
+                        vx = vg[off];
+                    }
                 }
                 kr[idx] = kx;
                 vr[idx] = vx;
             }
             __syncwarp();
+        }
+        if constexpr (kTMA && kGate && kMulti) {
+            // this chunk's r rows, read by its output pass a round later
+            if (lane == 0 && n > 0 && box_in(c0, t0 + warp * L, b))
+                tma_prefetch_3d_l2(&tmr, (int)c0, (int)(t0 + warp * L), b);
         }
         PairRef ref;
         St sum[2];
@@ -450,6 +533,10 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     //         [it % kAS][rank] of every CTA of the cluster, each store
     //         completing bytes on that CTA's barrier of the slot
     auto scan_push = [&](int round, int it) {
+        if (cta_failed()) return;
+#ifdef WKV4_CHECKED
+        if (p.no_push) return;
+#endif
         const TripleRef sums = triples(base + lay.sums(kMulti ? (round & 1) : 0), NW * Cg);
         const TripleRef agg = triples(base + lay.agg(it % kAS), NC * Cg);
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
@@ -492,16 +579,20 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
         const int as = it % kAS;
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
         const TripleRef agg = triples(base + lay.agg(as), NC * Cg);
-        if (!failed && !mbar_wait_cluster_bounded(abar + as, (uint32_t)((it / kAS) & 1))) {
-            failed = true;
-            if (lane == 0) atomicOr(&g_device_error, kErrExchangeWait);
-        }
         // The slot's next use is exchange it + 2.  Every CTA pushes it + 2
         // after its CTA barrier that follows its own fold of it + 1, which
         // waited for this CTA's push of it + 1, issued after the barrier
         // that follows this fold: the slot is read before it is overwritten,
-        // and re-armed (here) before it is written.
-        if (lane == 0 && it + kAS < items) mbar_arrive_expect_tx(abar + as, agg_bytes);
+        // and re-armed (here) before it is written.  A slot whose wait ran
+        // out (or was skipped after a failure) is not re-armed.
+        if (!cta_failed()) {
+            if (mbar_wait_cluster_bounded(abar + as, (uint32_t)((it / kAS) & 1), p.wait_rounds)) {
+                agg_waited = it + 1;
+                if (lane == 0 && it + kAS < items) mbar_arrive_expect_tx(abar + as, agg_bytes);
+            } else {
+                fail(kErrExchangeWait);
+            }
+        }
         const int64_t rrem = T - (t0 - (int64_t)rank * Ts);  // steps of the round from segment 0 on
         St P[2];
         switch (NC) {
@@ -548,28 +639,67 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     //         hold the next round's): y goes straight from registers, one
     //         2-channel store a step per lane (C % 4 == 0 with TMA, so a pair
     //         in range is whole and aligned).
-    auto emit = [&](int round, const PairRef& ref, const St (&S)[2]) {
+    auto emit = [&](int round, const PairRef& ref, const St (&S)[2], int phase) {
         const int slot = kMulti ? (round & 1) : 0;
         const int n = chunk_len(round, warp);
         const int64_t t0 = (int64_t)round * seg_stride + (int64_t)rank * Ts;
         const int64_t cpair = c0 + col;
-        const int64_t row0 = ((int64_t)b * T + t0 + warp * L) * C + cpair;  // k, v, y offset
+        const int64_t row0 = ((int64_t)b * T + t0 + warp * L) * C + cpair;  // k, v, y, r offset
         const bool ok0 = cpair < C, ok1 = cpair + 1 < C;
         IO* yrow = yg + row0;
+        const IO* rrow = rg + row0;  // kGate only
+        // every global access of the output pass is row0 + s C + j, s < n, j <= ok1;
+        // a warp with a lane outside skips the pass as a whole (its steps are
+        // warp-collective)
+#ifdef WKV4_CHECKED
+        const bool out_ok = !(ok0 && n > 0) || (in_range(row0, BTC) &&
+                                                in_range(row0 + (int64_t)(n - 1) * C + (ok1 ? 1 : 0), BTC));
+        if (!__all_sync(0xffffffffu, out_ok)) return;
+#endif
         auto out_one = [=](int s, int j, float y) {
-            if (j == 0 ? ok0 : ok1) yrow[(int64_t)s * C + j] = Io<IO>::from_f(y);
+            if (j == 0 ? ok0 : ok1) {
+                if constexpr (kGate) y = gate_one(y, Io<IO>::to_f(rrow[(int64_t)s * C + j]));
+                yrow[(int64_t)s * C + j] = Io<IO>::from_f(y);
+            }
         };
+        // g = e^{-r} of step s's pair from global memory (a pair whose first
+        // channel is in range is whole whenever C % 4 == 0, as with TMA)
+        auto gate_global = fn_gate([=](int s) -> f2 {
+            const IO* rp = rrow + (int64_t)s * C;
+            if (kTMA) return ok0 ? gate_g2(Pair<IO>::load(rp)) : 0ull;
+            const float r0 = ok0 ? Io<IO>::to_f(rp[0]) : 0.f, r1 = ok1 ? Io<IO>::to_f(rp[1]) : 0.f;
+            return gate_g2(pk(r0, r1));
+        });
         if constexpr (kTMA) {
             if constexpr (!kMulti) {
                 IO* yr = vr;
-                auto st_one = [=](int s, int j, float y) { yr[s * Cg + col + j] = Io<IO>::from_f(y); };
+                if constexpr (kGate) {
+                    // this warp's r rows (receptance barrier, phase `phase`)
+                    if (n > 0 && !cta_failed()) {
+                        if (mbar_wait_bounded(rbar + warp, (uint32_t)(phase & 1), p.wait_rounds)) {
+                            if (r_pend == phase) r_pend = -1;
+                        } else {
+                            fail(kErrTmaWait);
+                        }
+                    }
+                }
+                auto st_one = [=](int s, int j, float y) {
+                    if constexpr (kGate) y = gate_one(y, Io<IO>::to_f(yr[s * Cg + col + j]));
+                    yr[s * Cg + col + j] = Io<IO>::from_f(y);
+                };
                 auto st_pair = [=](int s, f2 y) { Pair<IO>::store(yr + s * Cg + col, y); };
-                chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
-                                          st_pair, st_one);
+                if constexpr (kGate) {
+                    auto gate_smem = fn_gate([=](int s) { return gate_g2(Pair<IO>::load(yr + s * Cg + col)); });
+                    chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0,
+                                              ok1, st_pair, st_one, gate_smem);
+                } else {
+                    chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0,
+                                              ok1, st_pair, st_one);
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    if (n > 0 && !failed) {
+                    if (n > 0 && !failed && box_in(c0, t0 + warp * L, b)) {
                         tma_store_3d(&tmy, yr, (int)c0, (int)(t0 + warp * L), b);
                         bulk_commit();
                     }
@@ -579,8 +709,13 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
                 auto out_pair = [=](int s, f2 y) {
                     if (ok0) Pair<IO>::store(yrow + (int64_t)s * C, y);
                 };
-                chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
-                                          out_pair, out_one);
+                if constexpr (kGate) {
+                    chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0,
+                                              ok1, out_pair, out_one, gate_global);
+                } else {
+                    chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0,
+                                              ok1, out_pair, out_one);
+                }
             }
         } else {
             // element-wise stores (any alignment)
@@ -588,8 +723,13 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
                 if (ok0) yrow[(int64_t)s * C] = Io<IO>::from_f(lo(y));
                 if (ok1) yrow[(int64_t)s * C + 1] = Io<IO>::from_f(hi(y));
             };
-            chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
-                                      out_pair, out_one);
+            if constexpr (kGate) {
+                chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
+                                          out_pair, out_one, gate_global);
+            } else {
+                chunk_phase3_stash<IO, L>(ref, n, S, cc, taddr(slot), kg + row0, vg + row0, C, ok0, ok1,
+                                          out_pair, out_one);
+            }
         }
     };
 
@@ -607,34 +747,44 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
         // only after barrier B of the tile that read them.
         for (int j = 0; j < items; ++j) {
             const bool more = j + 1 < items;
-            take_params(j & 1, (uint32_t)((j >> 1) & 1));
-            const PairRef ref = summary(0, (uint32_t)(j & 1));
+            take_params(j & 1, (uint32_t)((j >> 1) & 1), j);
+            const PairRef ref = summary(0, j);
             const int nt = tile + G, nb = nt / p.CGB;  // the next tile, if `more`
             const int64_t nc0 = (int64_t)(nt - nb * p.CGB) * Cg;
+            bool next_rows = false;  // this warp's rows of the next tile are on their way
             if (kTMA && more) {
                 __syncwarp();  // every lane has read the rows
-                if (lane == 0) {
-                    if (warp == 0) issue_params((j + 1) & 1, nb, nc0);
-                    issue_k(0, nb, nc0);
+                next_rows = __shfl_sync(0xffffffffu, lane == 0 && !cta_failed(), 0);
+                if (lane == 0 && next_rows) {
+                    if (warp == 0) issue_params((j + 1) & 1, nb, nc0, j + 1);
+                    issue_k(0, nb, nc0, j + 1);
                 }
             }
+            if constexpr (kTMA && kGate) {
+                // this tile's r rows into the v rows the summary pass has read
+                if (!(kTMA && more)) __syncwarp();
+                const bool go = __shfl_sync(0xffffffffu, lane == 0 && !cta_failed(), 0);
+                if (lane == 0 && go) issue_r(b, c0, j);
+            }
             __syncthreads();  // A: every summary of the tile is in
+            sync_fail();
             if (j == 0) cluster_wait();  // every CTA of the cluster has started
             if (warp == 0) scan_push(0, j);
             if (warp == 2) chunk_prefixes();
-            if (warp == 1) {
-                fold(0, j);
-                put_state_out();
-            }
+            if (warp == 1) fold(0, j);
             __syncthreads();  // B: the segment start state and the chunk prefixes are in place
+            sync_fail();
             const TripleRef st = triples(base + lay.start(0), Cg);
             const TripleRef pre = triples(base + lay.pre(), NW * Cg);
             St S[2];
 #pragma unroll
             for (int q = 0; q < 2; ++q)
                 S[q] = combine(st.get(col + q), pre.get(warp * Cg + col + q), (double)(warp * L) * cc.w2[q]);
-            emit(0, ref, S);
-            if (kTMA && more) {
+            emit(0, ref, S, j);
+            put_state_out();  // warp 1 (rank 0): the tile's final state, off the exchange's path
+            if (kTMA && next_rows) {
+                // issued whenever the k rows were, failure or not: the phase
+                // announced both
                 if (lane == 0) {
                     bulk_wait_read_all();  // the staged y has been read
                     issue_v(0, nb, nc0);
@@ -655,37 +805,52 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
         // round r, and warp 1 has folded round r; after it warp 0 scans and
         // pushes round r + 1, every warp emits round r, and warp 1 folds round
         // r + 1, whose aggregates have had a whole output pass to arrive.
-        take_params(0, 0);
+        take_params(0, 0, 0);
         PairRef ref_cur = summary(0, 0);
         if (kTMA && p.rounds > 1) {
             __syncwarp();  // every lane has read the rows
-            if (lane == 0) issue_rows(1, b, c0);
+            if (lane == 0 && !cta_failed()) issue_rows(1, b, c0, 1);
         }
         __syncthreads();  // every summary of round 0 is in
+        sync_fail();
         cluster_wait();   // every CTA of the cluster has started
         if (warp == 0) scan_push(0, 0);
         for (int round = 0; round < p.rounds; ++round) {
             const bool more = round + 1 < p.rounds;
             PairRef ref_next = ref_cur;
             if (more) {
-                ref_next = summary(round + 1, (uint32_t)((round + 1) & 1));
+                ref_next = summary(round + 1, round + 1);
                 if (kTMA && round + 2 < p.rounds) {
                     __syncwarp();  // every lane has read the rows
-                    if (lane == 0) issue_rows(round + 2, b, c0);
+                    if (lane == 0 && !cta_failed()) issue_rows(round + 2, b, c0, round + 2);
                 }
             }
             if (round == 0 && warp == 1) fold(0, 0);
             __syncthreads();
+            sync_fail();
             if (more && warp == 0) scan_push(round + 1, round + 1);
             St S[2];
             chunk_start(round, S);
-            emit(round, ref_cur, S);
+            emit(round, ref_cur, S, round);
             if (more && warp == 1) fold(round + 1, round + 1);
             ref_cur = ref_next;
         }
         put_state_out();
     }
 
+    // After a failure: let the copies this CTA issued and the aggregates its
+    // slots were armed for land before leaving (bounded waits; without a
+    // failure nothing is pending here).
+    if (kTMA && lane == 0 && row_pend >= 0)
+        mbar_wait_bounded(mbar + warp, (uint32_t)(row_pend & 1), p.wait_rounds);
+    if (kTMA && kGate && !kMulti && lane == 0 && r_pend >= 0)
+        mbar_wait_bounded(rbar + warp, (uint32_t)(r_pend & 1), p.wait_rounds);
+    if (kTMA && warp == 0 && lane == 0 && par_pend >= 0)
+        mbar_wait_bounded(pbar + (par_pend & 1), (uint32_t)((par_pend >> 1) & 1), p.wait_rounds);
+    if (warp == 1 && lane == 0) {
+        for (int e = agg_waited; e < agg_waited + kAS && e < items; ++e)
+            mbar_wait_cluster_bounded(abar + e % kAS, (uint32_t)((e / kAS) & 1), p.wait_rounds);
+    }
     // Every warp's tensor-memory accesses have completed (each load and each
     // store pass ends in its wait); release the columns.  No cluster barrier
     // is needed before leaving: every aggregate pushed into this CTA has

@@ -54,6 +54,9 @@ __global__ void __launch_bounds__(256) wkv4_token_shift_kernel(const ShiftParams
     const int64_t t0 = (int64_t)blockIdx.y * kShiftRun;
     const int64_t t1 = min(p.T, t0 + kShiftRun);
     const IO* x = static_cast<const IO*>(p.x);
+    // every access is (b T + t) C + c .. + V - 1 for t in [t0 - 1, t1), or a
+    // [B][C] row at b C + c (checked builds)
+    if (!in_range(c + V - 1, p.C) || !in_range(b, p.B) || !in_range(t1 - 1, p.T)) return;
     float xp[V], xt[V], o[V];
     if (t0 > 0) {
         load_vec<IO, V>(x + (b * p.T + t0 - 1) * p.C + c, xp);

@@ -12,6 +12,7 @@ Workloads (sizes of the RWKV-4 models the pages discuss):
   paradigm (WKV/RNN)", Methods table, "Model" and "Precision" rows).
 * ``rwkv4_14b_prefill``    B=4,  T=1024,  C=5120, bf16 I/O, zero state
   (d_model 5120 and 1K context of "RWKV-4 14B", "Every architecture field").
+* ``rwkv4_14b_prefill_gated``  the same with the receptance gate (r ~ N(0, 4)).
 * ``decode_b256``          B=256, C=5120, T=1 per call for 1024 calls, bf16.
 * ``decode_slots_b256``    the same calls, each serving 256 of a pool of 1024
   conversation states (slot-indexed decode; ids drawn per call).
@@ -69,6 +70,7 @@ class Workload:
     steps: int = 1                 # decode workloads: number of T=1 calls
     slots: int = 0                 # slot-indexed decode: states in the pool (0: one per row)
     op: str = "wkv"                # "wkv" or "token_shift"
+    gated: bool = False            # the gated forward (y = sigmoid(r) wkv; r from receptance())
 
     @property
     def channel_steps(self) -> int:
@@ -88,6 +90,8 @@ WORKLOADS = {
                                    seed=1, random_state=True),
     "rwkv4_14b_prefill": Workload("rwkv4_14b_prefill", B=4, T=1024, C=5120, dtype="bf16",
                                   seed=2, k_var=2.0),
+    "rwkv4_14b_prefill_gated": Workload("rwkv4_14b_prefill_gated", B=4, T=1024, C=5120,
+                                        dtype="bf16", seed=2, k_var=2.0, gated=True),
     "decode_b256": Workload("decode_b256", B=256, T=1, C=5120, dtype="bf16", seed=3,
                             steps=1024),
     "decode_slots_b256": Workload("decode_slots_b256", B=256, T=1, C=5120, dtype="bf16", seed=3,

@@ -26,8 +26,10 @@ STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_DTYPE", -3: "ERR_ALIAS", -4: "ERR_CUD
 
 _DTYPES = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
 
-EXPORTS = ("wkv4_decode_step", "wkv4_decode_step_slots", "wkv4_device_error", "wkv4_forward",
-           "wkv4_forward_variant", "wkv4_status_string", "wkv4_token_shift", "wkv4_version")
+EXPORTS = ("wkv4_decode_step", "wkv4_decode_step_gated", "wkv4_decode_step_slots",
+           "wkv4_device_error", "wkv4_forward", "wkv4_forward_gated", "wkv4_forward_gated_variant",
+           "wkv4_forward_variant", "wkv4_state_combine", "wkv4_status_string", "wkv4_token_shift",
+           "wkv4_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -56,6 +58,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.wkv4_forward_variant.restype = i32
             lib.wkv4_decode_step.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp, vp, i32]
             lib.wkv4_decode_step.restype = i32
+            gfwd = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32]
+            lib.wkv4_forward_gated.argtypes = gfwd
+            lib.wkv4_forward_gated.restype = i32
+            lib.wkv4_forward_gated_variant.argtypes = gfwd + [i32]
+            lib.wkv4_forward_gated_variant.restype = i32
+            lib.wkv4_decode_step_gated.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32]
+            lib.wkv4_decode_step_gated.restype = i32
+            lib.wkv4_state_combine.argtypes = [i64, i64, vp, i64, vp, vp, vp, vp]
+            lib.wkv4_state_combine.restype = i32
             lib.wkv4_decode_step_slots.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32]
             lib.wkv4_decode_step_slots.restype = i32
             lib.wkv4_token_shift.argtypes = [i64, i64, i64] + [vp] * 10 + [i32]
@@ -78,10 +89,32 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, device: Optional[torch.device] = None) -> ctypes.c_void_p:
+    """The call's stream: `stream`, or the current stream of `device`.  A torch
+    stream given for a call on `device` must belong to that device."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and isinstance(stream, torch.cuda.Stream) and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _one_device(**tensors) -> torch.device:
+    """The CUDA device all given tensors live on (None entries are skipped);
+    raises when they are spread over several devices.  The library launches
+    on the caller's current device, so every call runs with this device made
+    current."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, other arguments on {dev}")
+    return dev
 
 
 def _check_dev(name: str, t: Optional[torch.Tensor], dtype=None):
@@ -122,10 +155,52 @@ def forward(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
     if state_out is None and want_state:
         state_out = torch.empty((3, B, C), dtype=torch.float32, device=k.device)
     _check_dev("state_out", state_out, torch.float32)
-    rc = load().wkv4_forward_variant(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(state_in),
-                                     _ptr(y), _ptr(state_out), _stream(stream), dt, int(variant))
+    dev = _one_device(k=k, v=v, w=w, u=u, state_in=state_in, y=y, state_out=state_out)
+    with torch.cuda.device(dev):
+        rc = load().wkv4_forward_variant(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v),
+                                         _ptr(state_in), _ptr(y), _ptr(state_out),
+                                         _stream(stream, dev), dt, int(variant))
     if rc != 0:
         raise Wkv4Error(rc, "wkv4_forward")
+    return y, state_out
+
+
+def forward_gated(k: torch.Tensor, v: torch.Tensor, r: torch.Tensor, w: torch.Tensor,
+                  u: torch.Tensor, state_in: Optional[torch.Tensor] = None, *,
+                  y: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+                  want_state: bool = True, variant: int = KERNEL_AUTO,
+                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """wkv4_forward_gated: y = sigmoid(r) * wkv over k, v, r [B, T, C] (one
+    dtype); w, u [C] fp32; state_in [3, B, C] fp32 or None.  Returns
+    (y, state_out)."""
+    if k.dim() != 3 or v.shape != k.shape or r.shape != k.shape:
+        raise ValueError("k, v and r must all be [B, T, C]")
+    B, T, C = k.shape
+    dt = _DTYPES.get(k.dtype)
+    if dt is None or v.dtype != k.dtype or r.dtype != k.dtype:
+        raise ValueError(f"unsupported dtype {k.dtype}/{v.dtype}/{r.dtype}")
+    for name, t in (("k", k), ("v", v), ("r", r)):
+        _check_dev(name, t)
+    _check_dev("w", w, torch.float32)
+    _check_dev("u", u, torch.float32)
+    _check_dev("state_in", state_in, torch.float32)
+    if w.shape != (C,) or u.shape != (C,):
+        raise ValueError("w and u must be [C]")
+    if state_in is not None and state_in.shape != (3, B, C):
+        raise ValueError("state_in must be [3, B, C]")
+    if y is None:
+        y = torch.empty_like(k)
+    _check_dev("y", y, k.dtype)
+    if state_out is None and want_state:
+        state_out = torch.empty((3, B, C), dtype=torch.float32, device=k.device)
+    _check_dev("state_out", state_out, torch.float32)
+    dev = _one_device(k=k, v=v, r=r, w=w, u=u, state_in=state_in, y=y, state_out=state_out)
+    with torch.cuda.device(dev):
+        rc = load().wkv4_forward_gated_variant(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
+                                               _ptr(state_in), _ptr(y), _ptr(state_out),
+                                               _stream(stream, dev), dt, int(variant))
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_forward_gated")
     return y, state_out
 
 
@@ -157,10 +232,42 @@ def decode_step(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tens
     if y is None:
         y = torch.empty_like(k)
     _check_dev("y", y, k.dtype)
-    rc = load().wkv4_decode_step(B, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(state), _ptr(y),
-                                 _stream(stream), dt)
+    dev = _one_device(k=k, v=v, w=w, u=u, state=state, y=y)
+    with torch.cuda.device(dev):
+        rc = load().wkv4_decode_step(B, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(state),
+                                     _ptr(y), _stream(stream, dev), dt)
     if rc != 0:
         raise Wkv4Error(rc, "wkv4_decode_step")
+    return y
+
+
+def decode_step_gated(k: torch.Tensor, v: torch.Tensor, r: torch.Tensor, w: torch.Tensor,
+                      u: torch.Tensor, state: torch.Tensor, *, y: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """wkv4_decode_step_gated: k, v, r [B, C]; state [3, B, C] fp32 updated in
+    place.  Returns y = sigmoid(r) * wkv [B, C]."""
+    if k.dim() != 2 or v.shape != k.shape or r.shape != k.shape:
+        raise ValueError("k, v and r must all be [B, C]")
+    B, C = k.shape
+    dt = _DTYPES.get(k.dtype)
+    if dt is None or v.dtype != k.dtype or r.dtype != k.dtype:
+        raise ValueError(f"unsupported dtype {k.dtype}/{v.dtype}/{r.dtype}")
+    for name, t in (("k", k), ("v", v), ("r", r)):
+        _check_dev(name, t)
+    _check_dev("w", w, torch.float32)
+    _check_dev("u", u, torch.float32)
+    _check_dev("state", state, torch.float32)
+    if state.shape != (3, B, C):
+        raise ValueError("state must be [3, B, C]")
+    if y is None:
+        y = torch.empty_like(k)
+    _check_dev("y", y, k.dtype)
+    dev = _one_device(k=k, v=v, r=r, w=w, u=u, state=state, y=y)
+    with torch.cuda.device(dev):
+        rc = load().wkv4_decode_step_gated(B, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
+                                           _ptr(state), _ptr(y), _stream(stream, dev), dt)
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_decode_step_gated")
     return y
 
 
@@ -189,8 +296,11 @@ def decode_step_slots(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torc
     if y is None:
         y = torch.empty_like(k)
     _check_dev("y", y, k.dtype)
-    rc = load().wkv4_decode_step_slots(B, C, state_pool.shape[1], _ptr(w), _ptr(u), _ptr(k), _ptr(v),
-                                       _ptr(state_pool), _ptr(slot_ids), _ptr(y), _stream(stream), dt)
+    dev = _one_device(k=k, v=v, w=w, u=u, state_pool=state_pool, slot_ids=slot_ids, y=y)
+    with torch.cuda.device(dev):
+        rc = load().wkv4_decode_step_slots(B, C, state_pool.shape[1], _ptr(w), _ptr(u), _ptr(k),
+                                           _ptr(v), _ptr(state_pool), _ptr(slot_ids), _ptr(y),
+                                           _stream(stream, dev), dt)
     if rc != 0:
         raise Wkv4Error(rc, "wkv4_decode_step_slots")
     return y
@@ -216,14 +326,40 @@ def token_shift(x: torch.Tensor, mix_k: torch.Tensor, mix_v: torch.Tensor,
         _check_dev(name, t, x.dtype)
         if t is not None and t.shape != (B, C):
             raise ValueError(f"{name} must be [B, C]")
+    dev = _one_device(x=x, mix_k=mix_k, mix_v=mix_v, mix_r=mix_r, x_prev=x_prev, x_last=x_last)
     xk, xv = torch.empty_like(x), torch.empty_like(x)
     xr = torch.empty_like(x) if mix_r is not None else None
-    rc = load().wkv4_token_shift(B, T, C, _ptr(x), _ptr(x_prev), _ptr(mix_k), _ptr(mix_v),
-                                 _ptr(mix_r), _ptr(xk), _ptr(xv), _ptr(xr), _ptr(x_last),
-                                 _stream(stream), dt)
+    with torch.cuda.device(dev):
+        rc = load().wkv4_token_shift(B, T, C, _ptr(x), _ptr(x_prev), _ptr(mix_k), _ptr(mix_v),
+                                     _ptr(mix_r), _ptr(xk), _ptr(xv), _ptr(xr), _ptr(x_last),
+                                     _stream(stream, dev), dt)
     if rc != 0:
         raise Wkv4Error(rc, "wkv4_token_shift")
     return xk, xv, xr
+
+
+def state_combine(x: Optional[torch.Tensor], y: torch.Tensor, n_steps: int, w: torch.Tensor, *,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """wkv4_state_combine: the state x (or None: empty) followed by a segment
+    of n_steps steps whose state from the empty state is y; x, y, out
+    [3, B, C] fp32, w [C] fp32.  Returns out."""
+    if y.dim() != 3 or y.shape[0] != 3 or (x is not None and x.shape != y.shape):
+        raise ValueError("x and y must be [3, B, C]")
+    _, B, C = y.shape
+    for name, t in (("x", x), ("y", y), ("w", w)):
+        _check_dev(name, t, torch.float32)
+    if w.shape != (C,):
+        raise ValueError("w must be [C]")
+    if out is None:
+        out = torch.empty_like(y)
+    _check_dev("out", out, torch.float32)
+    dev = _one_device(x=x, y=y, w=w, out=out)
+    with torch.cuda.device(dev):
+        rc = load().wkv4_state_combine(B, C, _ptr(w), int(n_steps), _ptr(x), _ptr(y), _ptr(out),
+                                       _stream(stream, dev))
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_state_combine")
+    return out
 
 
 def device_error(reset: bool = True) -> int:

@@ -147,3 +147,35 @@ def test_binding_rejects_host_tensors_and_bad_shapes():
         wkv4.token_shift(k[0], w, w)
     with pytest.raises(ValueError, match="CUDA tensor"):
         wkv4.token_shift(k, w, w)
+
+
+def _gated(B=2, T=8, C=16, w=P, u=P + 0x1000, k=P + 0x10000, v=P + 0x20000, r=P + 0x60000,
+           si=None, y=P + 0x30000, so=None, dtype=wkv4.F32, variant=wkv4.KERNEL_AUTO):
+    return wkv4.load().wkv4_forward_gated_variant(B, T, C, w, u, k, v, r, si, y, so, None, dtype,
+                                                  variant)
+
+
+def test_gated_argument_checks():
+    assert _gated(B=-1) == -1 and _gated(T=-1) == -1
+    assert _gated(dtype=4) == -2 and _gated(variant=8) == -7
+    assert _gated(r=None) == -1                       # the receptance is required
+    assert _gated(B=0, r=None) == 0                   # ... unless there is nothing to do
+    assert _gated(y=P + 0x60000 + 64) == -3           # y over r
+    assert _gated(so=P + 0x60000) == -3               # the state over r
+    lib = wkv4.load()
+    d = lib.wkv4_decode_step_gated
+    assert d(2, 16, P, P + 0x1000, P + 0x10000, P + 0x20000, None, P + 0x40000, P + 0x30000,
+             None, 0) == -1                           # no r
+    assert d(2, 16, P, P + 0x1000, P + 0x10000, P + 0x20000, P + 0x30000 + 8, P + 0x40000,
+             P + 0x30000, None, 0) == -3              # y over r
+
+
+def test_binding_requires_one_device():
+    import types
+    a = types.SimpleNamespace(is_cuda=True, device="cuda:0")
+    b = types.SimpleNamespace(is_cuda=True, device="cuda:1")
+    assert wkv4._one_device(k=a, v=a, y=None) == "cuda:0"
+    with pytest.raises(ValueError, match="cuda:1"):
+        wkv4._one_device(k=a, v=b)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        wkv4._one_device(k=types.SimpleNamespace(is_cuda=False, device="cpu"))

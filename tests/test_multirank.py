@@ -31,7 +31,7 @@ def _worker(rank, world, port, out):
 def test_max_over_ranks_two_gloo_ranks():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn")
         assert dict(out) == {0: 15.0, 1: 15.0}

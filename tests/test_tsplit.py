@@ -67,7 +67,7 @@ def _worker(rank, world, port, out):
 @pytest.mark.parametrize("world", [2, 3])
 def test_tsplit_ranks_match_one_call(world):
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn")
         res = dict(out)
