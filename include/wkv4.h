@@ -240,10 +240,14 @@ WKV4_API int wkv4_state_combine(int64_t B, int64_t C, const float* w, int64_t n_
 /*
  * Device-side error word of the current device (bit 1: a bounded wait for a
  * TMA copy ran out; bit 2: a bounded wait for a cluster peer's partial state
- * ran out; bit 8: a slot-indexed decode row named a slot outside its pool).
- * Synchronises the device, reads the word, and clears it when `reset` is
- * non-zero.  Returns WKV4_OK when the word is zero, WKV4_ERR_TIMEOUT when a
- * wait ran out, else WKV4_ERR_SLOT when a slot id was out of range,
+ * ran out; bit 8: a slot-indexed decode row named a slot outside its pool;
+ * bit 16, bounds-checked builds only: an index outside its buffer).  One word
+ * per device and process, shared by every stream and call.  Synchronises the
+ * WHOLE device (cudaDeviceSynchronize: every stream, not only the caller's),
+ * reads the word, and clears it when `reset` is non-zero -- meant for tests
+ * and error paths, not for polling after every call.  Returns WKV4_OK when
+ * the word is zero, WKV4_ERR_TIMEOUT when a wait ran out, else WKV4_ERR_SLOT
+ * when a slot id was out of range (or an index was out of bounds), or
  * WKV4_ERR_CUDA when the read itself failed.
  */
 WKV4_API int wkv4_device_error(int reset);

@@ -160,10 +160,14 @@ __device__ __forceinline__ bool fast_ok(float kmax, float kmin, float u, float w
 
 // fp32 state buffers <-> kernel state.  On the way out the max is rounded to
 // fp32 and the rounding error d (natural units, |d| <= half an ulp of the
-// max) is folded into a and b as a e^d = a + a (e^d - 1), b likewise, with
-// e^d - 1 from expm1f (d itself to within its last bit while |d| is below
-// about 2^-12; a max of 10^5 nats, after a long decay with nothing new, has
-// |d| up to 2^-5, where the first-order d alone would be off by d^2 / 2).
+// max) is folded into a and b as a e^d = a + a (e^d - 1), b likewise.  While
+// |d| < 2^-12 (a max below 4096 nats in magnitude, the usual case) e^d - 1
+// is d to within its last bit, and d is used as it is; beyond (a max of 10^5
+// nats after a long decay with nothing new has |d| up to 2^-5, where d alone
+// would be off by d^2 / 2) e^d - 1 comes from expm1f.
+__device__ __forceinline__ float fold_factor(float d) {
+    return fabsf(d) < 0x1p-12f ? d : expm1f(d);
+}
 __device__ __forceinline__ St load_state_log2(const float* __restrict__ s, int64_t BC, int64_t ch) {
     return {s[ch], s[BC + ch], (double)s[2 * BC + ch] * kLog2eD};
 }
@@ -171,7 +175,7 @@ __device__ __forceinline__ St load_state_log2(const float* __restrict__ s, int64
 __device__ __forceinline__ void store_state_nat_d(float* __restrict__ s, int64_t BC, int64_t ch,
                                                   float a, float b, double p_nat) {
     const float pf = (float)p_nat;
-    const float d = expm1f((float)(p_nat - (double)pf));
+    const float d = fold_factor((float)(p_nat - (double)pf));
     s[ch] = fmaf(a, d, a);
     s[BC + ch] = fmaf(b, d, b);
     s[2 * BC + ch] = pf;

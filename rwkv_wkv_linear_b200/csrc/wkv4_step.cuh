@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(256) wkv4_decode_kernel(const StepParams p) {
         St s = {a[j], bb[j], (double)pp[j]};
         yy[j] = step_nat<kGate>(s, kk[j], vv[j], w[j], u[j], kGate ? rr[j] : 0.f);
         const float pf = (float)s.p;
-        const float d = expm1f((float)(s.p - (double)pf));  // fold the max's rounding into a, b
+        const float d = fold_factor((float)(s.p - (double)pf));  // fold the max's rounding into a, b
         a[j] = fmaf(s.a, d, s.a);
         bb[j] = fmaf(s.b, d, s.b);
         pp[j] = pf;
