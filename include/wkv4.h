@@ -238,6 +238,54 @@ WKV4_API int wkv4_state_combine(int64_t B, int64_t C, const float* w, int64_t n_
                                 wkv4_stream_t stream);
 
 /*
+ * The forward (or, with r, the gated forward) from HOST buffers: the
+ * activations come from host memory and the outputs go back to it, the
+ * copies overlapped with the kernels.  T is cut into chunks of chunk_steps
+ * steps (0: the library's choice, about a sixteenth of the input bytes and
+ * at least 16 MB of them); while the forward runs on chunk i, chunk i + 1's
+ * inputs are copied in and chunk i - 1's outputs copied out, on two streams
+ * of the call's own, and the chunks are forward calls chained through one
+ * device state: the state after a call is the next call's initial state
+ * ("An RNN that claims to match transformers, now in chatbot form", "The
+ * interesting bit"), so the result is that of one wkv4_forward (or
+ * wkv4_forward_gated) over the whole T, to the rounding of the fp32 state
+ * at each chunk boundary.
+ *   w, u         [C] fp32 DEVICE pointers (the layer's parameters).
+ *   k, v         [B][T][C] in `dtype`, HOST pointers (pinned memory lets the
+ *                copies overlap; pageable memory works, serialised).
+ *   r            [B][T][C] in `dtype` on the host, or NULL: the ungated
+ *                forward.
+ *   state_in     [3][B][C] fp32 on the host, or NULL for the empty state.
+ *   y            [B][T][C] in `dtype` on the host.
+ *   state_out    [3][B][C] fp32 on the host, or NULL; may equal state_in.
+ *   workspace    DEVICE memory of the current device, owned by the caller,
+ *                at least wkv4_forward_host_workspace(B, T, C, dtype,
+ *                r != NULL, chunk_steps) bytes, 16-byte aligned; it holds two
+ *                chunks' k, v (r) and y and the state, and must not overlap
+ *                any other argument.  Contents undefined after the call.
+ *   chunk_steps  steps a chunk, or 0.
+ * The call is asynchronous on `stream` like every call of the library: y and
+ * state_out are complete once `stream` has reached the point after the call
+ * (it waits for the call's last copy).  The library allocates no device
+ * memory.  B == 0 or C == 0: no-op; T == 0: state_out <- state_in (or the
+ * empty state, written through the workspace).  Returns WKV4_ERR_ARG for a
+ * NULL required pointer, negative sizes or a workspace that is too small,
+ * WKV4_ERR_ALIAS for overlapping outputs (as wkv4_forward), WKV4_ERR_DTYPE,
+ * WKV4_ERR_CUDA; the errors of the chained forward calls pass through.
+ */
+WKV4_API int wkv4_forward_host(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                               const void* k, const void* v, const void* r,
+                               const float* state_in, void* y, float* state_out,
+                               void* workspace, size_t workspace_bytes, int64_t chunk_steps,
+                               wkv4_stream_t stream, int dtype);
+
+/* Workspace bytes wkv4_forward_host needs for these sizes (gated: r given;
+ * with T == 0 the state's bytes), or 0 for B or C <= 0, T or chunk_steps < 0
+ * or an unknown dtype. */
+WKV4_API size_t wkv4_forward_host_workspace(int64_t B, int64_t T, int64_t C, int dtype, int gated,
+                                            int64_t chunk_steps);
+
+/*
  * Device-side error word of the current device (bit 1: a bounded wait for a
  * TMA copy ran out; bit 2: a bounded wait for a cluster peer's partial state
  * ran out; bit 8: a slot-indexed decode row named a slot outside its pool;

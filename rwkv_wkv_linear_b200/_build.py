@@ -17,7 +17,8 @@ LIB = os.path.join(PKG, "libwkv4.so")
 # the bounds-checked build (WKV4_CHECKED: every global index checked, fault
 # injection switches read from the environment), for the failure tests
 CHECKED_LIB = os.path.join(PKG, "libwkv4_checked.so")
-SOURCES = [os.path.join(CSRC, "wkv4_kernels.cu"), os.path.join(CSRC, "wkv4_api.cpp")]
+SOURCES = [os.path.join(CSRC, "wkv4_kernels.cu"), os.path.join(CSRC, "wkv4_api.cpp"),
+           os.path.join(CSRC, "wkv4_host.cpp")]
 
 
 def deps():

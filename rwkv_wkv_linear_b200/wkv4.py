@@ -28,6 +28,7 @@ _DTYPES = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
 
 EXPORTS = ("wkv4_decode_step", "wkv4_decode_step_gated", "wkv4_decode_step_slots",
            "wkv4_device_error", "wkv4_forward", "wkv4_forward_gated", "wkv4_forward_gated_variant",
+           "wkv4_forward_host", "wkv4_forward_host_workspace",
            "wkv4_forward_variant", "wkv4_state_combine", "wkv4_status_string", "wkv4_token_shift",
            "wkv4_version")
 
@@ -65,6 +66,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.wkv4_forward_gated_variant.restype = i32
             lib.wkv4_decode_step_gated.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32]
             lib.wkv4_decode_step_gated.restype = i32
+            lib.wkv4_forward_host.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                              ctypes.c_size_t, i64, vp, i32]
+            lib.wkv4_forward_host.restype = i32
+            lib.wkv4_forward_host_workspace.argtypes = [i64, i64, i64, i32, i32, i64]
+            lib.wkv4_forward_host_workspace.restype = ctypes.c_size_t
             lib.wkv4_state_combine.argtypes = [i64, i64, vp, i64, vp, vp, vp, vp]
             lib.wkv4_state_combine.restype = i32
             lib.wkv4_decode_step_slots.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32]
@@ -201,6 +207,70 @@ def forward_gated(k: torch.Tensor, v: torch.Tensor, r: torch.Tensor, w: torch.Te
                                                _stream(stream, dev), dt, int(variant))
     if rc != 0:
         raise Wkv4Error(rc, "wkv4_forward_gated")
+    return y, state_out
+
+
+def _check_host(name: str, t: Optional[torch.Tensor], dtype=None):
+    if t is None:
+        return
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+
+
+def host_workspace_bytes(B: int, T: int, C: int, dtype: torch.dtype, gated: bool = False,
+                         chunk_steps: int = 0) -> int:
+    """wkv4_forward_host_workspace: device bytes forward_host needs."""
+    return int(load().wkv4_forward_host_workspace(B, T, C, _DTYPES[dtype], int(gated),
+                                                  int(chunk_steps)))
+
+
+def forward_host(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
+                 state_in: Optional[torch.Tensor] = None, r: Optional[torch.Tensor] = None, *,
+                 y: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+                 want_state: bool = True, workspace: Optional[torch.Tensor] = None,
+                 chunk_steps: int = 0, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """wkv4_forward_host: the forward (gated when r is given) with k, v, r,
+    state_in, y and state_out in HOST memory (CPU tensors; pinned ones let the
+    copies overlap the kernels) and w, u [C] fp32 on the device; workspace is
+    a CUDA uint8 tensor of at least host_workspace_bytes(...) bytes (allocated
+    when None).  Asynchronous on the stream: synchronise it before reading y.
+    Returns (y, state_out)."""
+    if k.dim() != 3 or v.shape != k.shape or (r is not None and r.shape != k.shape):
+        raise ValueError("k, v (and r) must be [B, T, C]")
+    B, T, C = k.shape
+    dt = _DTYPES.get(k.dtype)
+    if dt is None or v.dtype != k.dtype or (r is not None and r.dtype != k.dtype):
+        raise ValueError(f"unsupported dtype {k.dtype}/{v.dtype}")
+    for name, t in (("k", k), ("v", v), ("r", r)):
+        _check_host(name, t)
+    _check_host("state_in", state_in, torch.float32)
+    _check_dev("w", w, torch.float32)
+    _check_dev("u", u, torch.float32)
+    if w.shape != (C,) or u.shape != (C,):
+        raise ValueError("w and u must be [C]")
+    if state_in is not None and state_in.shape != (3, B, C):
+        raise ValueError("state_in must be [3, B, C]")
+    if y is None:
+        y = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+    _check_host("y", y, k.dtype)
+    if state_out is None and want_state:
+        state_out = torch.empty((3, B, C), dtype=torch.float32, pin_memory=True)
+    _check_host("state_out", state_out, torch.float32)
+    dev = _one_device(w=w, u=u, workspace=workspace)
+    need = host_workspace_bytes(B, T, C, k.dtype, r is not None, chunk_steps)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check_dev("workspace", workspace)
+    with torch.cuda.device(dev):
+        rc = load().wkv4_forward_host(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
+                                      _ptr(state_in), _ptr(y), _ptr(state_out), _ptr(workspace),
+                                      workspace.numel(), int(chunk_steps), _stream(stream, dev), dt)
+    if rc != 0:
+        raise Wkv4Error(rc, "wkv4_forward_host")
     return y, state_out
 
 

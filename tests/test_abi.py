@@ -179,3 +179,50 @@ def test_binding_requires_one_device():
         wkv4._one_device(k=a, v=b)
     with pytest.raises(ValueError, match="CUDA tensor"):
         wkv4._one_device(k=types.SimpleNamespace(is_cuda=False, device="cpu"))
+
+
+def _host(B=2, T=64, C=16, w=P, u=P + 0x1000, k=P + 0x100000, v=P + 0x200000, r=None, si=None,
+          y=P + 0x300000, so=None, ws=P + 0x10000000, wsb=None, chunk=0, dtype=wkv4.F32):
+    lib = wkv4.load()
+    if wsb is None:
+        wsb = lib.wkv4_forward_host_workspace(B, T, C, dtype, int(r is not None), chunk)
+    return lib.wkv4_forward_host(B, T, C, w, u, k, v, r, si, y, so, ws, wsb, chunk, None, dtype)
+
+
+def test_host_forward_workspace_sizes():
+    lib = wkv4.load()
+    ws = lib.wkv4_forward_host_workspace
+    # two slots of k, v, y (gated: and r) of one chunk, and the state, each 256-byte aligned
+    io = 2 * 64 * 16 * 4
+    assert ws(2, 64, 16, wkv4.F32, 0, 0) == 2 * 3 * io + 512
+    assert ws(2, 64, 16, wkv4.F32, 1, 0) == 2 * 4 * io + 512
+    assert ws(2, 64, 16, wkv4.F32, 0, 16) == 2 * 3 * (io // 4) + 512
+    assert ws(2, 64, 16, wkv4.F16, 0, 16) == 2 * 3 * 1024 + 512
+    assert ws(2, 0, 16, wkv4.F32, 0, 0) == 512          # T == 0: the state only
+    assert ws(0, 64, 16, wkv4.F32, 0, 0) == 0
+    assert ws(2, -1, 16, wkv4.F32, 0, 0) == 0
+    assert ws(2, 64, 16, 9, 0, 0) == 0
+    assert ws(2, 64, 16, wkv4.F32, 0, -3) == 0
+    # the default chunk: about a sixteenth of the inputs, at least 16 MB of them
+    big = ws(1, 65536, 2048, wkv4.F32, 0, 0)
+    assert big == 2 * 3 * 4096 * 2048 * 4 + 3 * 2048 * 4
+    # 14B width (B=4, C=5120, bf16: 80 KB of inputs a step): 16 MB / 80 KB + 1 = 205 steps
+    assert ws(4, 1024, 5120, wkv4.BF16, 0, 0) == 2 * 3 * 4 * 205 * 5120 * 2 + 3 * 4 * 5120 * 4
+
+
+def test_host_forward_argument_checks():
+    assert _host(B=-1) == -1 and _host(T=-1) == -1 and _host(C=-1) == -1
+    assert _host(chunk=-1) == -1
+    assert _host(dtype=4) == -2
+    assert _host(B=0) == 0 and _host(C=0) == 0
+    for name in ("w", "u", "k", "v", "y", "ws"):
+        assert _host(**{name: None}) == -1, name
+    # a workspace one byte short
+    full = wkv4.load().wkv4_forward_host_workspace(2, 64, 16, wkv4.F32, 0, 0)
+    assert _host(wsb=full - 1) == -1
+    # y over k (2*64*16*4 = 8192 bytes), the state over y, the workspace over k
+    assert _host(y=P + 0x100000 + 4096) == -3
+    assert _host(so=P + 0x300000 + 64) == -3
+    assert _host(ws=P + 0x100000 + 16) == -3
+    # state_out partially over state_in (equal is allowed)
+    assert _host(si=P + 0x400000, so=P + 0x400000 + 8) == -3
