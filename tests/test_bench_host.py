@@ -28,3 +28,18 @@ def test_kernel_hash_ignores_comments_and_follows_code(tmp_path):
     assert bench.kernel_source_hash(str(copy)) == base
     f.write_text(text + "\nstatic const int unused_constant = 1;\n")
     assert bench.kernel_source_hash(str(copy)) != base
+
+
+def test_kernel_hash_leaves_out_the_host_pipeline(tmp_path):
+    """wkv4_host.cpp only chains the forward's calls: a change there keeps the
+    recorded kernel traffic valid; a change to the launchers does not."""
+    csrc = os.path.join(bench.ROOT, "rwkv_wkv_linear_b200", "csrc")
+    copy = tmp_path / "csrc"
+    shutil.copytree(csrc, copy)
+    base = bench.kernel_source_hash(str(copy))
+    f = copy / "wkv4_host.cpp"
+    f.write_text(f.read_text() + "\nstatic const int another_constant = 2;\n")
+    assert bench.kernel_source_hash(str(copy)) == base
+    g = copy / "wkv4_api.cpp"
+    g.write_text(g.read_text() + "\nstatic const int another_constant = 2;\n")
+    assert bench.kernel_source_hash(str(copy)) != base
