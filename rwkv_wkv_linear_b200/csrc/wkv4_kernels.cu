@@ -201,9 +201,19 @@ static size_t scan_smem_request(size_t bytes, int cols, int cta_regs) {
 }
 
 // Scan configuration per I/O type: steps per warp chunk (a warp's rows are
-// L steps x 64 channels).
-template <typename IO> struct ScanL { static constexpr int L = 32; };
-template <> struct ScanL<float> { static constexpr int L = 16; };
+// L steps x 64 channels), with one round (L) and with several (LM).  fp32
+// takes 16-step chunks in one round (two CTAs of 8 warps an SM) and 32-step
+// chunks over several rounds, where the round's exchange and fold are then
+// spread over twice the steps (measured on the 65536-step workload: 291
+// against 325 us a call).
+template <typename IO> struct ScanL {
+    static constexpr int L = 32;
+    static constexpr int LM = 32;
+};
+template <> struct ScanL<float> {
+    static constexpr int L = 16;
+    static constexpr int LM = 32;
+};
 
 constexpr int kNwChoices[2] = {8, 4};  // warps per CTA, in order of preference
 
@@ -307,28 +317,39 @@ static cudaError_t scan_ctas_per_sm(int nw, int nc, int& bps) {
     return cudaSuccess;
 }
 
-// Launch shape of the scan: warps per CTA (NW), cluster size (NC) and the
-// number of clusters.  8 warps per CTA wherever it fits.  When T fits in at
-// most 8 segments, one round with NC = segments (rounded up to a power of
-// two), and as many clusters as the GPU holds at once (at most one per
-// channel tile), each walking its share of the tiles; when T needs several
-// rounds, NC is the largest power of two whose grid of one cluster per tile
-// still fits in one wave (a second wave of CTAs that each walk all of T would
-// be costly).  WKV4_SCAN_NW / WKV4_SCAN_CLUSTER override NW / NC, and
+// Launch shape of the scan: warps per CTA (NW), cluster size (NC), the
+// number of clusters and the chunk length.  8 warps per CTA wherever it
+// fits.  When T fits in at most 8 segments of L-step chunks, one round with
+// NC = segments (rounded up to a power of two), and as many clusters as the
+// GPU holds at once (at most one per channel tile), each walking its share
+// of the tiles; when T needs several rounds, chunks of LM steps where T still
+// spans more than 8 of their segments (else L), and NC is the largest power
+// of two whose grid of one cluster per tile still fits in one wave (a second
+// wave of CTAs that each walk all of T would be costly).  WKV4_SCAN_NW / WKV4_SCAN_CLUSTER override NW / NC, and
 // WKV4_SCAN_WAVES=1 gives one cluster per tile with one round (tuning).
 struct ScanShape {
     int nw, nc, rounds;
     int64_t clusters;
+    bool long_chunks;  // several rounds with LM-step chunks
 };
 
-template <typename IO, int L, bool kTMA, bool kGate>
+template <typename IO, int L, int LM, bool kTMA, bool kGate>
 static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
     const int force_nw = scan_overrides().nw, force_nc = scan_overrides().nc;
     cudaError_t e = cudaSuccess;
     for (int i = 0; i < 2; ++i) {
         const int nw = kNwChoices[i];
         if (force_nw && nw != force_nw) continue;
-        const int64_t nseg = (T + (int64_t)nw * L - 1) / ((int64_t)nw * L);
+        const int64_t nseg1 = (T + (int64_t)nw * L - 1) / ((int64_t)nw * L);
+        const int64_t nsegm = (T + (int64_t)nw * LM - 1) / ((int64_t)nw * LM);
+        // several rounds of LM-step chunks where T spans more than a cluster of their segments
+        const bool lm = LM != L && nseg1 > kMaxCluster && nsegm > kMaxCluster;
+        const int64_t nseg = lm ? nsegm : nseg1;
+        auto per_sm = [&](bool multi, int c, int& bps) {
+            if (!multi) return scan_ctas_per_sm<IO, L, false, kTMA, kGate>(nw, c, bps);
+            return lm ? scan_ctas_per_sm<IO, LM, true, kTMA, kGate>(nw, c, bps)
+                      : scan_ctas_per_sm<IO, L, true, kTMA, kGate>(nw, c, bps);
+        };
         int nc = 1;
         if (force_nc == 1 || force_nc == 2 || force_nc == 4 || force_nc == 8) {
             nc = force_nc;
@@ -337,8 +358,7 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
         } else {
             for (int c = kMaxCluster; c > 1; c /= 2) {
                 int bps = 0, fit = 0;
-                if ((e = scan_ctas_per_sm<IO, L, true, kTMA, kGate>(nw, c, bps)) != cudaSuccess)
-                    return e;
+                if ((e = per_sm(true, c, bps)) != cudaSuccess) return e;
                 if ((e = clusters_fit(i, c, bps, fit)) != cudaSuccess) return e;
                 if ((int64_t)fit >= tiles) {
                     nc = c;
@@ -348,10 +368,9 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
         }
         const int64_t rounds = (nseg + nc - 1) / nc;
         if (rounds > (1ll << 30)) continue;
+        if (lm && rounds < 2) continue;  // (a forced cluster size that covers T: not this shape)
         int bps = 0;
-        e = rounds == 1 ? scan_ctas_per_sm<IO, L, false, kTMA, kGate>(nw, nc, bps)
-                        : scan_ctas_per_sm<IO, L, true, kTMA, kGate>(nw, nc, bps);
-        if (e != cudaSuccess) return e;
+        if ((e = per_sm(rounds > 1, nc, bps)) != cudaSuccess) return e;
         if (bps <= 0) continue;  // does not fit on an SM
         int64_t clusters = tiles;
         if (rounds == 1 && !scan_overrides().waves) {
@@ -359,7 +378,7 @@ static cudaError_t pick_scan_shape(int64_t tiles, int64_t T, ScanShape& out) {
             if ((e = clusters_fit(i, nc, bps, fit)) != cudaSuccess) return e;
             if (fit > 0 && fit < tiles) clusters = fit;
         }
-        out = {nw, nc, (int)rounds, clusters};
+        out = {nw, nc, (int)rounds, clusters, lm};
         return cudaSuccess;
     }
     return cudaErrorInvalidConfiguration;
@@ -403,7 +422,7 @@ static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const S
 
 template <typename IO, bool kTMA, bool kGate>
 static cudaError_t launch_scan_t(const FwdArgs& a, EncodeFn encode) {
-    constexpr int L = ScanL<IO>::L;
+    constexpr int L = ScanL<IO>::L, LM = ScanL<IO>::LM;
     ScanParams p{};
     p.T = a.T;
     p.C = a.C;
@@ -424,12 +443,15 @@ static cudaError_t launch_scan_t(const FwdArgs& a, EncodeFn encode) {
     const int64_t tiles = a.B * p.CGB;
     if (tiles > (1ll << 30)) return cudaErrorInvalidConfiguration;
     ScanShape sh;
-    cudaError_t e = pick_scan_shape<IO, L, kTMA, kGate>(tiles, a.T, sh);
+    cudaError_t e = pick_scan_shape<IO, L, LM, kTMA, kGate>(tiles, a.T, sh);
     if (e != cudaSuccess) return e;
     if (sh.clusters * sh.nc > (int64_t)INT32_MAX) return cudaErrorInvalidConfiguration;
     p.tiles = (int)tiles;
     p.rounds = sh.rounds;
     if (sh.rounds == 1) return launch_scan_nb<IO, L, false, kTMA, kGate>(a, p, sh, encode);
+    if constexpr (LM != L) {
+        if (sh.long_chunks) return launch_scan_nb<IO, LM, true, kTMA, kGate>(a, p, sh, encode);
+    }
     return launch_scan_nb<IO, L, true, kTMA, kGate>(a, p, sh, encode);
 }
 
