@@ -83,7 +83,7 @@ struct DeviceResources {
     std::mutex lock;
     bool ready = false;
     cudaStream_t in = nullptr, out = nullptr;
-    cudaEvent_t start = nullptr, end = nullptr;
+    cudaEvent_t start = nullptr, end = nullptr, in_done = nullptr;
     cudaEvent_t in_ready[2] = {nullptr, nullptr}, in_free[2] = {nullptr, nullptr};
     cudaEvent_t y_ready[2] = {nullptr, nullptr}, y_free[2] = {nullptr, nullptr};
     cudaError_t create() {
@@ -91,7 +91,7 @@ struct DeviceResources {
         cudaError_t e;
         if (!in && (e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking)) != cudaSuccess) return e;
         if (!out && (e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking)) != cudaSuccess) return e;
-        cudaEvent_t* all[] = {&start, &end, &in_ready[0], &in_ready[1], &in_free[0],
+        cudaEvent_t* all[] = {&start, &end, &in_done, &in_ready[0], &in_ready[1], &in_free[0],
                               &in_free[1], &y_ready[0], &y_ready[1], &y_free[0], &y_free[1]};
         for (cudaEvent_t* ev : all)
             if (!*ev && (e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
@@ -127,6 +127,80 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     if (!a || !b || !na || !nb) return false;
     const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
     return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+namespace {
+
+// The copies and forward calls of wkv4_forward_host, chunk by chunk, on the
+// device's copy streams and `cs` (see the top of the file); returns at the
+// first error, leaving what it queued to the caller's join.
+int issue_chunks(DeviceResources& res, int64_t B, int64_t T, int64_t C, const float* w,
+                 const float* u, const void* k, const void* v, const void* r,
+                 const float* state_in, void* y, float* state_out, const Plan& pl,
+                 unsigned char* ws, int dtype, cudaStream_t cs) {
+    const wkv4_stream_t stream = (wkv4_stream_t)cs;
+    const bool gated = r != nullptr;
+    const size_t es = dtype_bytes(dtype);
+    const size_t st_bytes = (size_t)3 * B * C * 4;
+    float* dstate = reinterpret_cast<float*>(ws + 2 * pl.slot);
+    auto slot_k = [&](int s) { return ws + (size_t)s * pl.slot; };
+    auto slot_v = [&](int s) { return slot_k(s) + pl.io; };
+    auto slot_y = [&](int s) { return slot_k(s) + 2 * pl.io; };
+    auto slot_r = [&](int s) { return slot_k(s) + 3 * pl.io; };
+    const size_t spitch = (size_t)T * C * es;  // a batch row of a host tensor
+    cudaError_t e;
+    // the copies follow whatever the caller queued on `stream` before
+    if ((e = cudaEventRecord(res.start, cs)) != cudaSuccess) return cuda_rc(e);
+    if ((e = cudaStreamWaitEvent(res.in, res.start, 0)) != cudaSuccess) return cuda_rc(e);
+    if ((e = cudaStreamWaitEvent(res.out, res.start, 0)) != cudaSuccess) return cuda_rc(e);
+    if (state_in &&
+        (e = cudaMemcpyAsync(dstate, state_in, st_bytes, cudaMemcpyDefault, res.in)) != cudaSuccess)
+        return cuda_rc(e);
+    const int64_t nchunks = (T + pl.tc - 1) / pl.tc;
+    for (int64_t i = 0; i < nchunks; ++i) {
+        const int s = (int)(i & 1);
+        const int64_t t0 = i * pl.tc, n = std::min(pl.tc, T - t0);
+        const size_t width = (size_t)n * C * es;  // a batch row of the chunk
+        const size_t off = (size_t)t0 * C * es;
+        // in (i)
+        if (i >= 2 && (e = cudaStreamWaitEvent(res.in, res.in_free[s], 0)) != cudaSuccess) return cuda_rc(e);
+        if ((e = copy_block(slot_k(s), width, static_cast<const unsigned char*>(k) + off, spitch, width,
+                            B, cudaMemcpyDefault, res.in)) != cudaSuccess)
+            return cuda_rc(e);
+        if ((e = copy_block(slot_v(s), width, static_cast<const unsigned char*>(v) + off, spitch, width,
+                            B, cudaMemcpyDefault, res.in)) != cudaSuccess)
+            return cuda_rc(e);
+        if (gated && (e = copy_block(slot_r(s), width, static_cast<const unsigned char*>(r) + off, spitch,
+                                     width, B, cudaMemcpyDefault, res.in)) != cudaSuccess)
+            return cuda_rc(e);
+        if ((e = cudaEventRecord(res.in_ready[s], res.in)) != cudaSuccess) return cuda_rc(e);
+        // run (i): chunk 0 starts from state_in (or the empty state), every
+        // later chunk from the state the one before left
+        if ((e = cudaStreamWaitEvent(cs, res.in_ready[s], 0)) != cudaSuccess) return cuda_rc(e);
+        if (i >= 2 && (e = cudaStreamWaitEvent(cs, res.y_free[s], 0)) != cudaSuccess) return cuda_rc(e);
+        const float* sin = (i == 0 && !state_in) ? nullptr : dstate;
+        const int rc = gated ? wkv4_forward_gated(B, n, C, w, u, slot_k(s), slot_v(s), slot_r(s), sin,
+                                                  slot_y(s), dstate, stream, dtype)
+                             : wkv4_forward(B, n, C, w, u, slot_k(s), slot_v(s), sin, slot_y(s), dstate,
+                                            stream, dtype);
+        if (rc != WKV4_OK) return rc;
+        if ((e = cudaEventRecord(res.in_free[s], cs)) != cudaSuccess) return cuda_rc(e);
+        if ((e = cudaEventRecord(res.y_ready[s], cs)) != cudaSuccess) return cuda_rc(e);
+        // out (i)
+        if ((e = cudaStreamWaitEvent(res.out, res.y_ready[s], 0)) != cudaSuccess) return cuda_rc(e);
+        if ((e = copy_block(static_cast<unsigned char*>(y) + off, spitch, slot_y(s), width, width, B,
+                            cudaMemcpyDefault, res.out)) != cudaSuccess)
+            return cuda_rc(e);
+        if ((e = cudaEventRecord(res.y_free[s], res.out)) != cudaSuccess) return cuda_rc(e);
+    }
+    // the final state leaves after the last chunk's kernels (the out stream
+    // waited for them)
+    if (state_out &&
+        (e = cudaMemcpyAsync(state_out, dstate, st_bytes, cudaMemcpyDefault, res.out)) != cudaSuccess)
+        return cuda_rc(e);
+    return WKV4_OK;
 }
 
 }  // namespace
@@ -187,12 +261,6 @@ int wkv4_forward_host(int64_t B, int64_t T, int64_t C, const float* w, const flo
         if (overlaps(workspace, pl.total, host[i], host_n[i])) return WKV4_ERR_ALIAS;
 
     unsigned char* ws = static_cast<unsigned char*>(workspace);
-    float* dstate = reinterpret_cast<float*>(ws + 2 * pl.slot);
-    auto slot_k = [&](int s) { return ws + (size_t)s * pl.slot; };
-    auto slot_v = [&](int s) { return slot_k(s) + pl.io; };
-    auto slot_y = [&](int s) { return slot_k(s) + 2 * pl.io; };
-    auto slot_r = [&](int s) { return slot_k(s) + 3 * pl.io; };
-    const size_t spitch = (size_t)T * C * es;  // a batch row of a host tensor
 
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -202,58 +270,15 @@ int wkv4_forward_host(int64_t B, int64_t T, int64_t C, const float* w, const flo
     std::lock_guard<std::mutex> guard(rp->lock);
     DeviceResources& res = *rp;
     if ((e = res.create()) != cudaSuccess) return cuda_rc(e);
-    // the copies follow whatever the caller queued on `stream` before
-    if ((e = cudaEventRecord(res.start, cs)) != cudaSuccess) return cuda_rc(e);
-    if ((e = cudaStreamWaitEvent(res.in, res.start, 0)) != cudaSuccess) return cuda_rc(e);
-    if ((e = cudaStreamWaitEvent(res.out, res.start, 0)) != cudaSuccess) return cuda_rc(e);
-    if (state_in &&
-        (e = cudaMemcpyAsync(dstate, state_in, st_bytes, cudaMemcpyDefault, res.in)) != cudaSuccess)
-        return cuda_rc(e);
-    const int64_t nchunks = (T + pl.tc - 1) / pl.tc;
-    for (int64_t i = 0; i < nchunks; ++i) {
-        const int s = (int)(i & 1);
-        const int64_t t0 = i * pl.tc, n = std::min(pl.tc, T - t0);
-        const size_t width = (size_t)n * C * es;  // a batch row of the chunk
-        const size_t off = (size_t)t0 * C * es;
-        // in (i)
-        if (i >= 2 && (e = cudaStreamWaitEvent(res.in, res.in_free[s], 0)) != cudaSuccess) return cuda_rc(e);
-        if ((e = copy_block(slot_k(s), width, static_cast<const unsigned char*>(k) + off, spitch, width,
-                            B, cudaMemcpyDefault, res.in)) != cudaSuccess)
-            return cuda_rc(e);
-        if ((e = copy_block(slot_v(s), width, static_cast<const unsigned char*>(v) + off, spitch, width,
-                            B, cudaMemcpyDefault, res.in)) != cudaSuccess)
-            return cuda_rc(e);
-        if (gated && (e = copy_block(slot_r(s), width, static_cast<const unsigned char*>(r) + off, spitch,
-                                     width, B, cudaMemcpyDefault, res.in)) != cudaSuccess)
-            return cuda_rc(e);
-        if ((e = cudaEventRecord(res.in_ready[s], res.in)) != cudaSuccess) return cuda_rc(e);
-        // run (i): chunk 0 starts from state_in (or the empty state), every
-        // later chunk from the state the one before left
-        if ((e = cudaStreamWaitEvent(cs, res.in_ready[s], 0)) != cudaSuccess) return cuda_rc(e);
-        if (i >= 2 && (e = cudaStreamWaitEvent(cs, res.y_free[s], 0)) != cudaSuccess) return cuda_rc(e);
-        const float* sin = (i == 0 && !state_in) ? nullptr : dstate;
-        const int rc = gated ? wkv4_forward_gated(B, n, C, w, u, slot_k(s), slot_v(s), slot_r(s), sin,
-                                                  slot_y(s), dstate, stream, dtype)
-                             : wkv4_forward(B, n, C, w, u, slot_k(s), slot_v(s), sin, slot_y(s), dstate,
-                                            stream, dtype);
-        if (rc != WKV4_OK) return rc;
-        if ((e = cudaEventRecord(res.in_free[s], cs)) != cudaSuccess) return cuda_rc(e);
-        if ((e = cudaEventRecord(res.y_ready[s], cs)) != cudaSuccess) return cuda_rc(e);
-        // out (i)
-        if ((e = cudaStreamWaitEvent(res.out, res.y_ready[s], 0)) != cudaSuccess) return cuda_rc(e);
-        if ((e = copy_block(static_cast<unsigned char*>(y) + off, spitch, slot_y(s), width, width, B,
-                            cudaMemcpyDefault, res.out)) != cudaSuccess)
-            return cuda_rc(e);
-        if ((e = cudaEventRecord(res.y_free[s], res.out)) != cudaSuccess) return cuda_rc(e);
-    }
-    // the final state leaves after the last chunk's kernels (the out stream
-    // waited for them)
-    if (state_out &&
-        (e = cudaMemcpyAsync(state_out, dstate, st_bytes, cudaMemcpyDefault, res.out)) != cudaSuccess)
-        return cuda_rc(e);
-    if ((e = cudaEventRecord(res.end, res.out)) != cudaSuccess) return cuda_rc(e);
-    if ((e = cudaStreamWaitEvent(cs, res.end, 0)) != cudaSuccess) return cuda_rc(e);
-    return WKV4_OK;
+    const int rc = issue_chunks(res, B, T, C, w, u, k, v, r, state_in, y, state_out, pl, ws, dtype, cs);
+    // `stream` waits for whatever this call queued on the copy streams -- after an error too, so
+    // that no copy of the call is still in flight once `stream` has passed it
+    cudaError_t e1 = cudaEventRecord(res.end, res.out);
+    if (e1 == cudaSuccess) e1 = cudaStreamWaitEvent(cs, res.end, 0);
+    cudaError_t e2 = cudaEventRecord(res.in_done, res.in);
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(cs, res.in_done, 0);
+    if (rc != WKV4_OK) return rc;
+    return cuda_rc(e1 != cudaSuccess ? e1 : e2);
 }
 
 }  // extern "C"

@@ -10,6 +10,12 @@ switch in the environment:
                                              N-th call's launch fails
                                              (WKV4_ERR_CUDA), every other
                                              call succeeds and is correct
+  python -m tests.failure_child host         with WKV4_FAULT=launch:2: the
+                                             forward from host buffers fails
+                                             at its second chunk's launch
+                                             (WKV4_ERR_CUDA), and the same call
+                                             repeated on the same workspace and
+                                             stream is correct
   python -m tests.failure_child exchange     with WKV4_FAULT=exchange: a scan
                                              call whose segment aggregates are
                                              never pushed ends with
@@ -37,7 +43,7 @@ def _dev(x):
     return {k: (t.to(DEV) if t is not None else None) for k, t in x.items()}
 
 
-def _check_fwd(x, dt, y, s, what, r=None):
+def _check_fwd(x, dt, y, s, what, r=None, calls=0):
     if r is None:
         y_ref, s_ref = oracle.forward(x["k"], x["v"], x["w"], x["u"], x["state_in"])
         ya = None if dt == "f32" else parity.y_abs(x["k"], x["v"], x["w"], x["u"], x["state_in"])
@@ -45,8 +51,9 @@ def _check_fwd(x, dt, y, s, what, r=None):
         y_ref, s_ref = oracle.forward_gated(x["k"], x["v"], r, x["w"], x["u"], x["state_in"])
         ya = None if dt == "f32" else parity.y_abs_gated(x["k"], x["v"], r, x["w"], x["u"],
                                                          x["state_in"])
-    parity.check_y(y.cpu(), y_ref, x["v"], dt, what + " y", y_abs=ya)
-    parity.check_state(s.cpu(), s_ref, x["v"], x["state_in"], what=what + " state")
+    parity.check_y(y.cpu(), y_ref, x["v"], dt, what + " y", y_abs=ya, calls=calls)
+    parity.check_state(s.cpu(), s_ref, x["v"], x["state_in"], calls=max(1, calls),
+                       what=what + " state")
 
 
 # one call of every entry point, on small valid shapes
@@ -153,6 +160,24 @@ def main():
                     raise AssertionError(f"call {i} ({call.__name__}) did not fail")
             else:
                 call()
+        assert wkv4.device_error(reset=True) == 0
+    elif mode == "host":
+        assert os.environ.get("WKV4_FAULT") == "launch:2"
+        x = synth.custom(2, 900, 128, "bf16", seed=8, random_state=True, k_var=2.0)
+        w, u = x["w"].to(DEV), x["u"].to(DEV)
+        kh, vh, sh = x["k"].pin_memory(), x["v"].pin_memory(), x["state_in"].pin_memory()
+        ws = torch.empty(wkv4.host_workspace_bytes(2, 900, 128, torch.bfloat16, chunk_steps=300),
+                         dtype=torch.uint8, device=DEV)
+        try:
+            wkv4.forward_host(kh, vh, w, u, sh, workspace=ws, chunk_steps=300)
+        except wkv4.Wkv4Error as e:
+            assert e.status == -4, e.status  # WKV4_ERR_CUDA
+        else:
+            raise AssertionError("the injected launch failure did not surface")
+        torch.cuda.synchronize()
+        y, s = wkv4.forward_host(kh, vh, w, u, sh, workspace=ws, chunk_steps=300)
+        torch.cuda.synchronize()
+        _check_fwd(x, "bf16", y, s, "host after the failure", calls=3)
         assert wkv4.device_error(reset=True) == 0
     elif mode == "exchange":
         assert os.environ.get("WKV4_FAULT") == "exchange"

@@ -9,6 +9,9 @@ process of its own (tests/failure_child.py):
 * host-side fault injection (WKV4_FAULT=launch:N): the N-th launch is made
   with an empty grid, which the runtime rejects without running anything; the
   call returns WKV4_ERR_CUDA and every other call succeeds;
+* the forward from host buffers whose second chunk's launch is made to fail
+  returns WKV4_ERR_CUDA with its queued copies joined into the caller's
+  stream, and the same call repeated is correct;
 * a bounded device wait that runs out (WKV4_FAULT=exchange, a short limit):
   no scan CTA pushes its segment aggregate, on a shape of one channel tile and
   one round, so that no copy and no DSMEM store is in flight when the waits
@@ -54,6 +57,10 @@ def test_checked_build_records_nothing_on_valid_shapes(checked_lib):
 @pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 6])
 def test_injected_launch_failure(checked_lib, n):
     _child("launch", str(n), WKV4_FAULT=f"launch:{n}")
+
+
+def test_host_forward_launch_failure(checked_lib):
+    _child("host", WKV4_FAULT="launch:2")
 
 
 def test_exchange_wait_runs_out(checked_lib):
