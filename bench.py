@@ -31,6 +31,13 @@ drawn per call.
 (wkv4_token_shift: B=4, T=1024, C=5120, bf16, three outputs); a step is one
 call, the metric counts B*T*C elements as channel-steps.
 
+``e2e`` is the same metric end to end from host memory: for the prefill
+workloads one wkv4_forward_host call a step (pinned host buffers in, y and
+the state out, the copies in both directions overlapped with the kernels in
+chunks of T); for the decode and token-shift workloads the step's inputs are
+copied in from pinned host memory, the call made and its outputs copied out,
+on one stream.
+
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead
 (rank 0 only; other ranks exit).
 """
