@@ -290,7 +290,7 @@ int wkv4_token_shift(int64_t B, int64_t T, int64_t C, const void* x, const void*
         return cuda_status(e);
     }
     if (!x || !mix_k || !mix_v || !xk || !xv || (mix_r && !xr)) return WKV4_ERR_ARG;
-    if (B > 65535 || T > 65535ll * 16) return WKV4_ERR_ARG;  // grid z (rows), y (runs of 16 steps)
+    if (B > 65535 || T > 65535ll * 16) return WKV4_ERR_ARG;  // grid z (rows), y (at most 65535 runs)
     if (!mix_r) xr = nullptr;
     const Range in[5] = {range_of(x, io), range_of(x_prev, row), range_of(mix_k, C * 4),
                          range_of(mix_v, C * 4), range_of(mix_r, mix_r ? C * 4 : 0)};

@@ -88,7 +88,7 @@ constexpr int kMaxDevices = 64;
 // device (the launchers run on every call; attribute queries are not free).
 struct DeviceAttrs {
     int smem_per_sm = 233472, smem_reserved = 1024, reg_file = 65536, max_threads = 2048,
-        max_blocks = 32;
+        max_blocks = 32, sms = 148;
 };
 
 static const DeviceAttrs& device_attrs() {
@@ -107,6 +107,7 @@ static const DeviceAttrs& device_attrs() {
         cudaDeviceGetAttribute(&a.reg_file, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
         cudaDeviceGetAttribute(&a.max_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
         cudaDeviceGetAttribute(&a.max_blocks, cudaDevAttrMaxBlocksPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&a.sms, cudaDevAttrMultiProcessorCount, dev);
         cudaGetLastError();
     });
     return attrs[dev];
@@ -603,6 +604,43 @@ cudaError_t launch_decode_slots(const FwdArgs& a, const int32_t* slots, int64_t 
     return cudaGetLastError();
 }
 
+// CTAs of one token-shift instantiation an SM holds (the runtime's occupancy
+// query, once per device).
+template <typename IO, int V>
+static int shift_ctas_per_sm() {
+    static std::atomic<int> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 1;
+    }
+    int n = cache[dev].load(std::memory_order_acquire);
+    if (n == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, wkv4_token_shift_kernel<IO, V>,
+                                                          kShiftThreads, 0) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = 1;
+        }
+        cache[dev].store(n, std::memory_order_release);
+    }
+    return n;
+}
+
+template <typename IO, int V>
+static void launch_shift_t(ShiftParams& p, int64_t groups, cudaStream_t stream) {
+    // one wave: runs = the CTAs the GPU holds over the CTAs a step range
+    // needs (channel blocks x batch rows), at least kShiftMinRun steps a run
+    // and at most 65535 runs
+    const int64_t xb = (groups + kShiftThreads - 1) / kShiftThreads;
+    const int64_t slots = (int64_t)device_attrs().sms * shift_ctas_per_sm<IO, V>();
+    const int64_t runs = std::max<int64_t>(1, slots / std::max<int64_t>(1, xb * p.B));
+    int64_t run = std::max<int64_t>((p.T + runs - 1) / runs, kShiftMinRun);
+    run = std::max<int64_t>(run, (p.T + 65534) / 65535);
+    p.run = run;
+    const dim3 grid((unsigned)xb, (unsigned)((p.T + run - 1) / run), (unsigned)p.B);
+    wkv4_token_shift_kernel<IO, V><<<launch_grid(grid), kShiftThreads, 0, stream>>>(p);
+}
+
 cudaError_t launch_token_shift(const ShiftArgs& a) {
     ShiftParams p{};
     p.B = a.B;
@@ -620,19 +658,17 @@ cudaError_t launch_token_shift(const ShiftArgs& a) {
     bool vec = a.C % V == 0 && aligned(a.x, 16) && aligned(a.x_prev, 16) && aligned(a.x_last, 16);
     for (int i = 0; i < 3; ++i) vec = vec && aligned(a.mix[i], 16) && aligned(a.out[i], 16);
     const int64_t groups = (a.C + (vec ? V : 1) - 1) / (vec ? V : 1);
-    const dim3 grid((unsigned)((groups + 255) / 256), (unsigned)((a.T + kShiftRun - 1) / kShiftRun),
-                    (unsigned)a.B);
     if (vec) {
         switch (a.dtype) {
-            case WKV4_F32: wkv4_token_shift_kernel<float, 4><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
-            case WKV4_F16: wkv4_token_shift_kernel<__half, 8><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
-            default: wkv4_token_shift_kernel<__nv_bfloat16, 8><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            case WKV4_F32: launch_shift_t<float, 4>(p, groups, a.stream); break;
+            case WKV4_F16: launch_shift_t<__half, 8>(p, groups, a.stream); break;
+            default: launch_shift_t<__nv_bfloat16, 8>(p, groups, a.stream); break;
         }
     } else {
         switch (a.dtype) {
-            case WKV4_F32: wkv4_token_shift_kernel<float, 1><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
-            case WKV4_F16: wkv4_token_shift_kernel<__half, 1><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
-            default: wkv4_token_shift_kernel<__nv_bfloat16, 1><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            case WKV4_F32: launch_shift_t<float, 1>(p, groups, a.stream); break;
+            case WKV4_F16: launch_shift_t<__half, 1>(p, groups, a.stream); break;
+            default: launch_shift_t<__nv_bfloat16, 1>(p, groups, a.stream); break;
         }
     }
     return cudaGetLastError();

@@ -7,9 +7,11 @@
 // three mix vectors (k, v, r) in one pass over x.
 //
 // An HBM stream: each thread owns V channels (16 bytes) of one batch row and
-// walks a run of kRun steps, keeping the previous token in registers, so x is
-// read once (plus one row per run) and each output written once.  Computed in
-// fp32 as x_prev + mix (x - x_prev) and rounded once to the I/O type.
+// walks a run of steps, keeping the previous token in registers, so x is read
+// once (plus one row per run) and each output written once.  The launcher
+// sizes the runs so that the grid is one wave of the CTAs the GPU holds at
+// once (no tail of a second, partial wave).  Computed in fp32 as
+// x_prev + mix (x - x_prev) and rounded once to the I/O type.
 #pragma once
 
 #include "wkv4_device.cuh"
@@ -23,9 +25,11 @@ struct ShiftParams {
     const float* mix[3];  // k, v, r; r may be null
     void* out[3];        // xk, xv, xr (xr null when mix r is)
     void* x_last;        // [B][C] or null
+    int64_t run;         // steps a thread walks
 };
 
-constexpr int kShiftRun = 16;  // steps a thread walks
+constexpr int kShiftThreads = 128;  // threads a CTA: channel groups of 128 V
+constexpr int kShiftMinRun = 8;     // shortest run (each run reads one row twice)
 
 // V fp32 values from p (16-byte pieces when V > 1).
 template <int V>
@@ -44,15 +48,16 @@ __device__ __forceinline__ void load_f32(const float* p, float (&o)[V]) {
     }
 }
 
-// grid: x = channel groups of 256 V, y = runs of kShiftRun steps, z = batch rows.
-// The caller checks that C % V == 0 and every pointer is 16-byte aligned when V > 1.
+// grid: x = channel groups of kShiftThreads V, y = runs of p.run steps, z =
+// batch rows.  The caller checks that C % V == 0 and every pointer is 16-byte
+// aligned when V > 1.
 template <typename IO, int V>
-__global__ void __launch_bounds__(256) wkv4_token_shift_kernel(const ShiftParams p) {
+__global__ void __launch_bounds__(kShiftThreads) wkv4_token_shift_kernel(const ShiftParams p) {
     const int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
     if (c >= p.C) return;
     const int64_t b = blockIdx.z;
-    const int64_t t0 = (int64_t)blockIdx.y * kShiftRun;
-    const int64_t t1 = min(p.T, t0 + kShiftRun);
+    const int64_t t0 = (int64_t)blockIdx.y * p.run;
+    const int64_t t1 = min(p.T, t0 + p.run);
     const IO* x = static_cast<const IO*>(p.x);
     // every access is (b T + t) C + c .. + V - 1 for t in [t0 - 1, t1), or a
     // [B][C] row at b C + c (checked builds)
