@@ -51,6 +51,19 @@ __device__ __forceinline__ bool in_range(int64_t i, int64_t n) {
 __device__ __forceinline__ constexpr bool in_range(int64_t, int64_t) { return true; }
 #endif
 
+// Programmatic dependent launch.  Every kernel of the library is launched so
+// that it may start while the kernel before it in the stream is finishing
+// (its CTAs become resident and set up as the earlier grid's CTAs leave); it
+// lets the next one do the same as soon as it starts, and touches no global
+// memory before grid_dependency_wait(), which returns once the earlier grid
+// has completed and its memory is visible (at once for a normal launch).
+__device__ __forceinline__ void allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr double kLog2eD = 1.4426950408889634;
 constexpr double kLn2D = 0.6931471805599453;

@@ -113,6 +113,26 @@ static const DeviceAttrs& device_attrs() {
     return attrs[dev];
 }
 
+// A launch that may begin while the kernel before it in the stream is
+// finishing (programmatic stream serialization): every kernel of the library
+// waits for the earlier grid before its first global access.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Tuning overrides of the scan's launch shape, read from the environment
 // once per process: WKV4_SCAN_NW (warps per CTA), WKV4_SCAN_CLUSTER (cluster
 // size), WKV4_SCAN_WAVES=1 (one cluster per channel tile with one round).
@@ -411,13 +431,15 @@ static cudaError_t launch_scan_nb(const FwdArgs& a, const ScanParams& p, const S
     cfg.blockDim = dim3(32 * sh.nw, 1, 1);
     cfg.dynamicSmemBytes = scan_smem_request(lay.bytes(), lay.tmem_cols(), warp_regs(regs) * sh.nw);
     cfg.stream = a.stream;
-    cudaLaunchAttribute attrs[1];
+    cudaLaunchAttribute attrs[2];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
     attrs[0].val.clusterDim.x = (unsigned)sh.nc;
     attrs[0].val.clusterDim.y = 1;
     attrs[0].val.clusterDim.z = 1;
+    attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, tk, tv, ty, tr, p);
 }
 
@@ -491,7 +513,9 @@ static cudaError_t launch_seq_g(const FwdArgs& a, const CUtensorMap* tk, const C
     p.BC = a.B * a.C;
     p.wait_rounds = wait_rounds();
     const int64_t grid = a.B * p.CGB;
-    kern<<<launch_grid((unsigned)grid), Sh::kThreads, Sh::kSmem, a.stream>>>(*tk, *tv, *tr, p);
+    e = launch_pdl(kern, dim3(launch_grid((unsigned)grid)), dim3(Sh::kThreads), Sh::kSmem, a.stream, *tk, *tv,
+                   *tr, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -529,10 +553,11 @@ static StepParams step_params(const FwdArgs& a) {
 
 template <typename IO>
 static void launch_step_io(const FwdArgs& a, const StepParams& p, unsigned grid) {
+    const dim3 g(launch_grid(grid));
     if (a.r)
-        wkv4_step_kernel<IO, true><<<launch_grid(grid), 256, 0, a.stream>>>(p);
+        launch_pdl(wkv4_step_kernel<IO, true>, g, dim3(256), 0, a.stream, p);
     else
-        wkv4_step_kernel<IO, false><<<launch_grid(grid), 256, 0, a.stream>>>(p);
+        launch_pdl(wkv4_step_kernel<IO, false>, g, dim3(256), 0, a.stream, p);
 }
 
 cudaError_t launch_step(const FwdArgs& a) {
@@ -551,12 +576,16 @@ static bool aligned(const void* ptr, size_t bytes) {
     return ptr == nullptr || ((uintptr_t)ptr % bytes) == 0;
 }
 
-template <typename IO, int V>
+// (kSlots: the slot-indexed decode, which has no gate)
+template <typename IO, int V, bool kSlots = false>
 static void launch_decode_io(const FwdArgs& a, const StepParams& p, unsigned grid) {
-    if (a.r)
-        wkv4_decode_kernel<IO, V, false, true><<<launch_grid(grid), 256, 0, a.stream>>>(p);
+    const dim3 g(launch_grid(grid));
+    if (kSlots)
+        launch_pdl(wkv4_decode_kernel<IO, V, true>, g, dim3(256), 0, a.stream, p);
+    else if (a.r)
+        launch_pdl(wkv4_decode_kernel<IO, V, false, true>, g, dim3(256), 0, a.stream, p);
     else
-        wkv4_decode_kernel<IO, V, false, false><<<launch_grid(grid), 256, 0, a.stream>>>(p);
+        launch_pdl(wkv4_decode_kernel<IO, V, false, false>, g, dim3(256), 0, a.stream, p);
 }
 
 cudaError_t launch_decode(const FwdArgs& a) {
@@ -590,15 +619,15 @@ cudaError_t launch_decode_slots(const FwdArgs& a, const int32_t* slots, int64_t 
     const unsigned grid = (unsigned)((threads + 255) / 256);
     if (vec) {
         switch (a.dtype) {
-            case WKV4_F32: wkv4_decode_kernel<float, V, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
-            case WKV4_F16: wkv4_decode_kernel<__half, V, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
-            default: wkv4_decode_kernel<__nv_bfloat16, V, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            case WKV4_F32: launch_decode_io<float, V, true>(a, p, grid); break;
+            case WKV4_F16: launch_decode_io<__half, V, true>(a, p, grid); break;
+            default: launch_decode_io<__nv_bfloat16, V, true>(a, p, grid); break;
         }
     } else {
         switch (a.dtype) {
-            case WKV4_F32: wkv4_decode_kernel<float, 1, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
-            case WKV4_F16: wkv4_decode_kernel<__half, 1, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
-            default: wkv4_decode_kernel<__nv_bfloat16, 1, true><<<launch_grid(grid), 256, 0, a.stream>>>(p); break;
+            case WKV4_F32: launch_decode_io<float, 1, true>(a, p, grid); break;
+            case WKV4_F16: launch_decode_io<__half, 1, true>(a, p, grid); break;
+            default: launch_decode_io<__nv_bfloat16, 1, true>(a, p, grid); break;
         }
     }
     return cudaGetLastError();
@@ -638,7 +667,7 @@ static void launch_shift_t(ShiftParams& p, int64_t groups, cudaStream_t stream) 
     run = std::max<int64_t>(run, (p.T + 65534) / 65535);
     p.run = run;
     const dim3 grid((unsigned)xb, (unsigned)((p.T + run - 1) / run), (unsigned)p.B);
-    wkv4_token_shift_kernel<IO, V><<<launch_grid(grid), kShiftThreads, 0, stream>>>(p);
+    launch_pdl(wkv4_token_shift_kernel<IO, V>, launch_grid(grid), dim3(kShiftThreads), 0, stream, p);
 }
 
 cudaError_t launch_token_shift(const ShiftArgs& a) {
@@ -677,16 +706,16 @@ cudaError_t launch_token_shift(const ShiftArgs& a) {
 cudaError_t launch_copy_state(const FwdArgs& a) {
     const int64_t BC = a.B * a.C;
     if (!a.state_out || BC == 0) return cudaSuccess;
-    wkv4_copy_state_kernel<<<launch_grid((unsigned)((BC + 255) / 256)), 256, 0, a.stream>>>(a.state_in,
-                                                                               a.state_out, BC);
+    const dim3 grid(launch_grid((unsigned)((BC + 255) / 256)));
+    launch_pdl(wkv4_copy_state_kernel, grid, dim3(256), 0, a.stream, a.state_in, a.state_out, BC);
     return cudaGetLastError();
 }
 
 cudaError_t launch_state_combine(int64_t B, int64_t C, const float* w, int64_t n, const float* x,
                                  const float* y, float* out, cudaStream_t stream) {
     const int64_t BC = B * C;
-    wkv4_state_combine_kernel<<<launch_grid((unsigned)((BC + 255) / 256)), 256, 0, stream>>>(
-        w, n, x, y, out, B, C);
+    const dim3 grid(launch_grid((unsigned)((BC + 255) / 256)));
+    launch_pdl(wkv4_state_combine_kernel, grid, dim3(256), 0, stream, w, n, x, y, out, B, C);
     return cudaGetLastError();
 }
 

@@ -245,6 +245,8 @@ __global__ void __maxnreg__((scan_maxnreg<L, kMulti>()))
     wkv4_scan_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const __grid_constant__ CUtensorMap tmy, const __grid_constant__ CUtensorMap tmr,
                      const ScanParams p) {
+    allow_dependents();
+    grid_dependency_wait();
     using Lay = ScanLayout<IO, L, kMulti>;
     constexpr int kAS = Lay::kAggSlots;
     constexpr int Cg = Lay::kCg;

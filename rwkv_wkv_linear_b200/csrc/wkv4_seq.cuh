@@ -40,6 +40,8 @@ template <typename IO, int L, int NW, int NS, bool kGate>
 __global__ void __launch_bounds__(32 * NW)
     wkv4_seq_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                     const __grid_constant__ CUtensorMap tmr, const SeqParams p) {
+    allow_dependents();
+    grid_dependency_wait();
     using Sh = SeqShape<IO, L, NW, NS>;
     constexpr int Cw = Sh::kCw;
     extern __shared__ unsigned char smem_raw[];

@@ -53,6 +53,8 @@ __device__ __forceinline__ void load_f32(const float* p, float (&o)[V]) {
 // aligned when V > 1.
 template <typename IO, int V>
 __global__ void __launch_bounds__(kShiftThreads) wkv4_token_shift_kernel(const ShiftParams p) {
+    allow_dependents();
+    grid_dependency_wait();
     const int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
     if (c >= p.C) return;
     const int64_t b = blockIdx.z;

@@ -30,6 +30,8 @@ struct StepParams {
 // kGate: y = sigmoid(r) wkv, the receptance gate of the time mix.
 template <typename IO, bool kGate = false>
 __global__ void __launch_bounds__(256) wkv4_step_kernel(const StepParams p) {
+    allow_dependents();
+    grid_dependency_wait();
     const int64_t BC = p.B * p.C;
     const int64_t ch = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (ch >= BC) return;
@@ -56,6 +58,8 @@ __global__ void __launch_bounds__(256) wkv4_step_kernel(const StepParams p) {
 // vector width.
 template <typename IO, int V, bool kSlots = false, bool kGate = false>
 __global__ void __launch_bounds__(256) wkv4_decode_kernel(const StepParams p) {
+    allow_dependents();
+    grid_dependency_wait();
     const int64_t BC = p.B * p.C;
     const int64_t ch = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
     if (ch >= BC) return;
@@ -122,6 +126,8 @@ __global__ void __launch_bounds__(256) wkv4_decode_kernel(const StepParams p) {
 __global__ void __launch_bounds__(256)
     wkv4_state_combine_kernel(const float* __restrict__ w, int64_t n, const float* x,
                               const float* y, float* out, int64_t B, int64_t C) {
+    allow_dependents();
+    grid_dependency_wait();
     const int64_t BC = B * C;
     const int64_t ch = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (ch >= BC) return;
@@ -139,6 +145,8 @@ __global__ void __launch_bounds__(256)
 }
 
 __global__ void __launch_bounds__(256) wkv4_copy_state_kernel(const float* in, float* out, int64_t BC) {
+    allow_dependents();
+    grid_dependency_wait();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= BC) return;
     if (in) {
