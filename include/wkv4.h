@@ -30,6 +30,15 @@
  * alignment: misaligned or odd-C inputs take a slower element-wise path.
  * NaN / Inf inputs propagate unchecked.  Distinct calls may run concurrently
  * on different streams.
+ *
+ * Every kernel is launched with programmatic stream serialization: it may
+ * start while the kernel before it on the stream is finishing, and touches no
+ * memory before that kernel has completed (griddepcontrol.wait); it lets the
+ * next kernel start at once (griddepcontrol.launch_dependents).  Ordering on
+ * the stream is unchanged for ordinary launches; a caller's own kernel
+ * launched with programmatic serialization right after a call must, as with
+ * any such launch, wait for the grid before it (cudaGridDependencySynchronize)
+ * before reading the call's outputs.
  */
 #ifndef WKV4_H
 #define WKV4_H
